@@ -101,6 +101,10 @@ static void init_formats(void)
  * is the saturating behaviour. */
 static int nearest_code(double a, const double* mags, int ncodes)
 {
+    /* saturating: at or above the largest value (this also keeps huge inputs,
+     * whose distances to the top two values round to the same double, on the
+     * largest code) */
+    if (a >= mags[ncodes - 1]) return ncodes - 1;
     int best = 0;
     double bd = fabs(a - mags[0]);
     for (int c = 1; c < ncodes; c++) {

@@ -78,7 +78,7 @@ def test_e4m3_rounding_matches_torch():
     mine = np.array([orc.e4m3_code(float(x)) for x in xs])
     assert np.array_equal(ref, mine)
     # saturation above the largest finite value
-    for x in (449.0, 464.0, 500.0, 1e9):
+    for x in (449.0, 464.0, 500.0, 1e9, 1e30, 3e38):
         assert orc.e4m3_code(x) == 0x7E
 
 
