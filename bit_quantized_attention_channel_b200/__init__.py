@@ -1,1 +1,199 @@
-"""B200-native NVFP4 attention (placeholder; the binding is added with the C-ABI)."""
+"""B200-native NVFP4 attention: Python binding of libsa (include/sa.h).
+
+This module only marshals arguments: it allocates result tensors with torch
+(device memory and streams are torch's plumbing) and passes raw pointers to the
+C ABI, whose CUDA kernels do every step of the computation.  There is no CPU or
+PyTorch fallback: if libsa.so is missing or a call fails, an exception is
+raised.
+
+Entry points keep the C names:
+  sa_quant_nvfp4        smoothing + NVFP4 pre-pass (max-scaling or ScaleSearch)
+  sa_thrift_select      high-precision block selector
+  sa_attn_fwd           NVFP4 attention forward (optionally with bf16 blocks)
+  sa_attn_decode_kvfp4  decode over an NVFP4 KV cache
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsa.so")
+
+SA_ROLE = {"q": 0, "k": 1, "v": 2}
+SA_SCALE = {"max": 0, "search": 1}
+STATUS = ["SA_OK", "SA_ERR_INVALID_ARG", "SA_ERR_UNSUPPORTED", "SA_ERR_WORKSPACE", "SA_ERR_NONFINITE", "SA_ERR_CUDA",
+          "SA_ERR_TIMEOUT", "SA_ERR_DEVICE_ASSERT"]
+
+
+class SAError(RuntimeError):
+    def __init__(self, fn, code):
+        name = STATUS[code] if 0 <= code < len(STATUS) else str(code)
+        super().__init__(f"{fn} returned {name}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libsa.so (built in-tree by build.py); raises if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libsa.so not found at {LIB_PATH}; run `python -m bit_quantized_attention_channel_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.sa_status_string.argtypes, L.sa_status_string.restype = [I], ctypes.c_char_p
+        L.sa_device_status.argtypes, L.sa_device_status.restype = [P, I], I
+        for n in ("sa_codes_bytes", "sa_scales_bytes"):
+            getattr(L, n).argtypes, getattr(L, n).restype = [I, I, I, I, I], Z
+        L.sa_quant_workspace_size.argtypes, L.sa_quant_workspace_size.restype = [I, I, I, I, I], Z
+        L.sa_quant_nvfp4.argtypes = [P, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, Z, P]
+        L.sa_quant_nvfp4.restype = I
+        L.sa_select_workspace_size.argtypes, L.sa_select_workspace_size.restype = [I, I, I, I], Z
+        L.sa_thrift_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P, Z, P]
+        L.sa_thrift_select.restype = I
+        L.sa_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, P, P, P, P, P, P]
+        L.sa_attn_fwd.restype = I
+        L.sa_decode_workspace_size.argtypes, L.sa_decode_workspace_size.restype = [I, I, I, I, I], Z
+        L.sa_attn_decode_kvfp4.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, P]
+        L.sa_attn_decode_kvfp4.restype = I
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise SAError(fn, code)
+
+
+def _empty(nbytes, device, dtype=None):
+    import torch
+
+    return torch.empty(max(int(nbytes), 1), dtype=dtype or torch.uint8, device=device)
+
+
+@dataclass
+class NVFP4Tensor:
+    """NVFP4 encoding of one [B,H,N,D] tensor (device memory).  codes and
+    scales use the layouts documented in include/sa.h."""
+    codes: "torch.Tensor"
+    scales: "torch.Tensor"
+    g: "torch.Tensor"  # float32[2] = {g, 1/g}
+    role: str
+    shape: tuple
+    k_mean: "torch.Tensor | None" = None
+    ss_off: "torch.Tensor | None" = None
+
+
+def sa_device_status(reset: bool = True, stream=None) -> int:
+    """Synchronise and return the library's device status word."""
+    return lib().sa_device_status(_stream(stream), int(reset))
+
+
+def sa_quant_nvfp4(x, role: str, smooth: bool = True, mode: str = "max", f_lo: int = -2, f_hi: int = 6,
+                   ss_offsets: bool = False, out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """Quantise bf16 x [B,H,N,D] (CUDA) to NVFP4 (see include/sa.h)."""
+    import torch
+
+    B, H, N, D = x.shape
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    L = lib()
+    r = SA_ROLE[role]
+    if out is None:
+        codes = _empty(L.sa_codes_bytes(B, H, N, D, r), x.device)
+        scales = _empty(L.sa_scales_bytes(B, H, N, D, r), x.device)
+        g = torch.empty(2, dtype=torch.float32, device=x.device)
+        km = torch.empty(B, H, D, dtype=torch.float32, device=x.device) if (r == 1 and smooth) else None
+        nblk = B * H * N * D // 16
+        off = torch.empty(max(nblk, 1), dtype=torch.int8, device=x.device) if ss_offsets else None
+        out = NVFP4Tensor(codes, scales, g, role, (B, H, N, D), km, off)
+    ws_bytes = L.sa_quant_workspace_size(B, H, N, D, r)
+    ws = _empty(ws_bytes, x.device)
+    _check("sa_quant_nvfp4",
+           L.sa_quant_nvfp4(_ptr(x), B, H, N, D, r, int(smooth), SA_SCALE[mode], f_lo, f_hi, _ptr(out.codes),
+                            _ptr(out.scales), _ptr(out.g), _ptr(out.k_mean), _ptr(out.ss_off), _ptr(ws), ws_bytes,
+                            _stream(stream)))
+    return out
+
+
+def sa_thrift_select(q, k, causal: bool, frac_bp: int = 500, stream=None):
+    """(mask uint8 [B,H,T,T], nsel int32 [B,H]) on the device."""
+    import torch
+
+    B, H, N, D = q.shape
+    T = (N + 127) // 128
+    L = lib()
+    mask = torch.empty(B, H, T, T, dtype=torch.uint8, device=q.device)
+    nsel = torch.empty(B, H, dtype=torch.int32, device=q.device)
+    ws_bytes = L.sa_select_workspace_size(B, H, N, D)
+    ws = _empty(ws_bytes, q.device)
+    _check("sa_thrift_select", L.sa_thrift_select(_ptr(q), _ptr(k), B, H, N, D, int(causal), int(frac_bp), _ptr(mask),
+                                                  _ptr(nsel), _ptr(ws), ws_bytes, _stream(stream)))
+    return mask, nsel
+
+
+def sa_attn_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, causal: bool, sm_scale: float = 0.0, mask=None,
+                q_bf16=None, k_bf16=None, v_bf16=None, want_lse: bool = False, out=None, stream=None):
+    """FP32 attention output [B,H,N,D] (and lse [B,H,N] if asked)."""
+    import torch
+
+    B, H, N, D = q.shape
+    dev = q.codes.device
+    if out is None:
+        out = torch.empty(B, H, N, D, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
+    km = k.k_mean if mask is not None else None
+    _check("sa_attn_fwd",
+           lib().sa_attn_fwd(_ptr(q.codes), _ptr(q.scales), _ptr(q.g), _ptr(k.codes), _ptr(k.scales), _ptr(k.g),
+                             _ptr(v.codes), _ptr(v.scales), _ptr(v.g), B, H, N, D, int(causal), float(sm_scale),
+                             _ptr(mask), _ptr(q_bf16), _ptr(k_bf16), _ptr(v_bf16), _ptr(km), _ptr(out), _ptr(lse),
+                             _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.0, out=None, stream=None):
+    """q bf16 [B,Hq,D]; caches quantised as [B,Hkv,L,D]; returns FP32 [B,Hq,D]."""
+    import torch
+
+    B, Hq, D = q.shape
+    _, Hkv, Lk, _ = k.shape
+    L = lib()
+    if out is None:
+        out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
+    ws_bytes = L.sa_decode_workspace_size(B, Hq, Hkv, Lk, D)
+    ws = _empty(ws_bytes, q.device)
+    _check("sa_attn_decode_kvfp4",
+           L.sa_attn_decode_kvfp4(_ptr(q), _ptr(k.codes), _ptr(k.scales), _ptr(k.g), _ptr(v.codes), _ptr(v.scales),
+                                  _ptr(v.g), B, Hq, Hkv, Lk, D, float(sm_scale), _ptr(out), _ptr(ws), ws_bytes,
+                                  _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------- layouts
+def scales_to_logical(scales, B: int, H: int, N: int, D: int, role: str):
+    """Unpack the tensor-core atom layout of scale bytes (include/sa.h) into
+    the logical row-major [B,H,R,C/16] layout (R, C = N, D for Q/K and D, N for
+    V).  Pure index permutation, host or device tensors."""
+    import torch
+
+    R, C = (D, N) if role == "v" else (N, D)
+    RT, CK = math.ceil(R / 128), math.ceil(C / 64)
+    a = scales.reshape(B * H, RT, CK, 32, 4, 4)  # [bh, rt, ck, r%32, r/32, j]
+    a = a.permute(0, 1, 4, 3, 2, 5)  # [bh, rt, r/32, r%32, ck, j]
+    a = a.reshape(B * H, RT * 128, CK * 4)[:, :R, : C // 16]
+    return a.reshape(B, H, R, C // 16).contiguous() if isinstance(a, torch.Tensor) else a

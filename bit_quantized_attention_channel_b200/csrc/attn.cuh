@@ -1,0 +1,293 @@
+// attn.cuh -- NVFP4 attention forward on tcgen05 block-scaled MMAs.
+//
+// "Search Your Block Floating Point Scales!" (gist.science summary),
+// "ScaleSearchAttention / 네이티브 NVFP4 실행": Q K^T and P V run natively in
+// NVFP4 on tensor cores with FP32 accumulation.  SageAttention3 article
+// (dasgeld.co): FP4 tensor-core attention on Blackwell.
+//
+// One CTA per (b, h, 128-query tile); thread i of the 128 owns query row i,
+// which is TMEM lane i of every accumulator.  Per key tile of 128:
+//   TMA K codes (128 x D/2 B, swizzled) + K scale atoms, V^T codes (D x 64 B)
+//   + V scale atoms -> tcgen05.cp scale atoms into TMEM ->
+//   S = Q K^T (kind::mxf4nvf4, M=128 N=128, D/64 MMAs of K=64) ->
+//   softmax rows from TMEM: running max m (log2 units), P~ = exp2(S c - m),
+//   per 16 keys: scale = E4M3(max p / 6) with p = 2688 P~, codes = E2M1(p/s)
+//   computed as exp2(S c + log2(2688) - m - log2 s) ->
+//   P codes to shared memory (64-byte swizzle, the MMA A layout), P scales to
+//   an atom -> rescale O and l in TMEM when the running max moved ->
+//   O += P V^T (N = D) and l += P 1 (N = 16, a constant all-ones operand), so
+//   l sums the dequantised P exactly on the tensor core.
+// Epilogue: out = O / l * g_V (FP32), lse = m ln2 + ln(l / 2688).
+#pragma once
+
+#include "tc.cuh"
+
+namespace sa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2_2688 = 11.392317422778761f;
+
+struct AttnParams {
+    const uint8_t* q_sf;
+    const uint8_t* k_sf;
+    const uint8_t* v_sf;
+    const float* q_g;
+    const float* k_g;
+    const float* v_g;
+    float* out;
+    float* lse;
+    int N, H;
+    int T;    // 128-row tiles of Q/K (= scale row tiles per (b,h))
+    int CKv;  // 64-key chunks of the V scale atoms per (b,h)
+    int causal;
+    float sm_scale;
+};
+
+template <int D>
+struct AttnSmem {
+    uint8_t q[128 * D / 2];   // Q tile, K-major, D/2-byte swizzle
+    uint8_t k[128 * D / 2];   // K tile
+    uint8_t v[D * 64];        // V^T tile: D rows x 128 keys, 64-byte swizzle
+    uint8_t p[128 * 64];      // P tile: 128 rows x 128 keys, 64-byte swizzle
+    uint8_t ones[16 * 64];    // constant operand: 16 rows of E2M1 1.0
+    uint8_t qsf[D / 64 * 512];
+    uint8_t ksf[D / 64 * 512];
+    uint8_t vsf[2 * 512];
+    uint8_t psf[2 * 512];
+    uint8_t onesf[512];
+    uint64_t tma_bar;
+    uint64_t mma_bar;
+    uint32_t tmem_slot;
+};
+
+// TMEM columns (512 allocated)
+constexpr uint32_t TM_S = 0, TM_O = 128, TM_L = 256, TM_SFQ = 272, TM_SFK = 280, TM_SFP = 288, TM_SFV = 296,
+                   TM_SF1 = 304;
+
+SA_DEV float tmem_ld1_sync(uint32_t taddr)
+{
+    uint32_t r;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r)
+        : "r"(taddr)
+        : "memory");
+    return __uint_as_float(r);
+}
+
+template <int D>
+SA_DEV bool attn_body(AttnSmem<D>& s, const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                      const AttnParams& p, int t, int bh, uint32_t tbase)
+{
+    constexpr int KB = D / 64;             // K=64 MMA steps for Q K^T
+    constexpr uint32_t QSW = D == 128 ? 4u : 6u;  // 64B / 32B swizzle
+    constexpr uint32_t QSBO = 8 * D / 2;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int row = t * 128 + tid;
+    const float c2 = p.q_g[0] * p.k_g[0] * p.sm_scale * kLog2e;
+    uint32_t tma_phase = 0, mma_phase = 0;
+
+    if (tid == 0) {
+        mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512);
+        tma_load_3d(s.q, tm_q, &s.tma_bar, 0, t * 128, bh);
+        bulk_load(s.qsf, p.q_sf + ((size_t)bh * p.T + t) * KB * 512, KB * 512, &s.tma_bar);
+    }
+    if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
+    tma_phase ^= 1;
+    if (tid == 0) {
+        tc_fence_after();
+        for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + TM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
+        tc_cp_sf(tbase + TM_SF1, smem_u32(s.onesf));
+    }
+
+    float m2 = -INFINITY;
+    const int Tk = (p.N + 127) / 128;
+    const int nt = p.causal ? min(t + 1, Tk) : Tk;
+    for (int u = 0; u < nt; u++) {
+        const int nk = min(128, p.N - u * 128);
+        const int kblocks = nk > 64 ? 2 : 1;
+        if (tid == 0) {
+            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
+            tma_load_3d(s.k, tm_k, &s.tma_bar, 0, u * 128, bh);
+            bulk_load(s.ksf, p.k_sf + ((size_t)bh * p.T + u) * KB * 512, KB * 512, &s.tma_bar);
+            tma_load_3d(s.v, tm_v, &s.tma_bar, u * 64, 0, bh);
+            bulk_load(s.vsf, p.v_sf + ((size_t)bh * p.CKv + 2 * u) * 512, kblocks * 512, &s.tma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
+        tma_phase ^= 1;
+        if (tid == 0) {
+            tc_fence_after();
+            for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + TM_SFK + 4 * kb, smem_u32(s.ksf + 512 * kb));
+            for (int kb = 0; kb < kblocks; kb++) tc_cp_sf(tbase + TM_SFV + 4 * kb, smem_u32(s.vsf + 512 * kb));
+            for (int kb = 0; kb < KB; kb++)
+                mma_fp4(tbase + TM_S, make_sdesc(smem_u32(s.q) + 32 * kb, QSBO, 16, QSW),
+                        make_sdesc(smem_u32(s.k) + 32 * kb, QSBO, 16, QSW), idesc_fp4(128, 128),
+                        tbase + TM_SFQ + 4 * kb, tbase + TM_SFK + 4 * kb, kb > 0);
+            tc_commit(&s.mma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // ---- this row's 128 scores
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+            tmem_ld32(tbase + lane_off + TM_S + 32 * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
+        tmem_wait_ld();
+        reg_fence(sv);
+
+        const int kbase = u * 128;
+        float bmax[8];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int blk = 0; blk < 8; blk++) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int j = kbase + blk * 16 + i;
+                const bool valid = j < p.N && (!p.causal || j <= row);
+                const float v = valid ? sv[blk * 16 + i] : -INFINITY;
+                sv[blk * 16 + i] = v;
+                mx = fmaxf(mx, v);
+            }
+            bmax[blk] = mx;
+            tmax = fmaxf(tmax, mx);
+        }
+        const float m2_new = fmaxf(m2, tmax * c2);
+        const float msub = m2_new == -INFINITY ? 0.0f : m2_new;
+        const float alpha = ex2f(m2 - msub);
+        uint32_t codes[16];
+        uint32_t scw0 = 0, scw1 = 0;
+#pragma unroll
+        for (int blk = 0; blk < 8; blk++) {
+            const float pmax = ex2f(fmaf(bmax[blk], c2, kLog2_2688 - msub));
+            const uint32_t sc = f32_to_e4m3(pmax * (1.0f / 6.0f));
+            const float bias = sc ? (kLog2_2688 - msub - lg2f(e4m3_to_f32(sc))) : -INFINITY;
+            float y[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) y[i] = ex2f(fmaf(sv[blk * 16 + i], c2, bias));
+            codes[2 * blk] = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+            codes[2 * blk + 1] = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+            if (blk < 4)
+                scw0 |= sc << (8 * blk);
+            else
+                scw1 |= sc << (8 * (blk - 4));
+        }
+        m2 = m2_new;
+
+        // ---- P codes (A operand, 64-byte swizzle) and scale atoms
+        uint8_t* prow = s.p + (tid >> 3) * 512 + (tid & 7) * 64;
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const int cs = c ^ ((tid & 7) >> 1);
+            *reinterpret_cast<uint4*>(prow + cs * 16) =
+                make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
+        }
+        *reinterpret_cast<uint32_t*>(s.psf + (tid & 31) * 16 + (tid >> 5) * 4) = scw0;
+        *reinterpret_cast<uint32_t*>(s.psf + 512 + (tid & 31) * 16 + (tid >> 5) * 4) = scw1;
+
+        // ---- rescale the accumulators when this warp's running max moved
+        if (u > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; c++) {
+                float o[32];
+                tmem_ld32(tbase + lane_off + TM_O + 32 * c, o);
+                tmem_wait_ld();
+                reg_fence(o);
+#pragma unroll
+                for (int i = 0; i < 32; i++) o[i] *= alpha;
+                tmem_st32(tbase + lane_off + TM_O + 32 * c, o);
+            }
+            const float l = tmem_ld1_sync(tbase + lane_off + TM_L);
+            tmem_st1(tbase + lane_off + TM_L, l * alpha);
+            tmem_wait_st();
+        }
+
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            for (int kb = 0; kb < kblocks; kb++) tc_cp_sf(tbase + TM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
+            for (int kb = 0; kb < kblocks; kb++) {
+                const uint64_t pd = make_sdesc(smem_u32(s.p) + 32 * kb, 512, 16, 4);
+                const uint32_t acc = (u > 0 || kb > 0) ? 1u : 0u;
+                mma_fp4(tbase + TM_O, pd, make_sdesc(smem_u32(s.v) + 32 * kb, 512, 16, 4), idesc_fp4(128, D),
+                        tbase + TM_SFP + 4 * kb, tbase + TM_SFV + 4 * kb, acc);
+                mma_fp4(tbase + TM_L, pd, make_sdesc(smem_u32(s.ones) + 32 * kb, 512, 16, 4), idesc_fp4(128, 16),
+                        tbase + TM_SFP + 4 * kb, tbase + TM_SF1, acc);
+            }
+            tc_commit(&s.mma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        mma_phase ^= 1;
+        tc_fence_after();
+    }
+
+    // ---- epilogue: out = O / l * g_V
+    const float l = tmem_ld1_sync(tbase + lane_off + TM_L);
+    const float scale = p.v_g[0] / l;
+    float* orow = p.out + ((size_t)bh * p.N + row) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; c++) {
+        float o[32];
+        tmem_ld32(tbase + lane_off + TM_O + 32 * c, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        if (row < p.N) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(orow + 32 * c + i) =
+                    make_float4(o[i] * scale, o[i + 1] * scale, o[i + 2] * scale, o[i + 3] * scale);
+        }
+    }
+    if (p.lse && row < p.N) p.lse[(size_t)bh * p.N + row] = m2 * kLn2 + logf(l * (1.0f / 2688.0f));
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 1) attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                          const __grid_constant__ CUtensorMap tm_k,
+                                                          const __grid_constant__ CUtensorMap tm_v,
+                                                          const AttnParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    AttnSmem<D>& s = *reinterpret_cast<AttnSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                     ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int t = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // long rows first
+    const int bh = blockIdx.z * p.H + blockIdx.y;
+
+    if (warp == 0) {
+        tmem_alloc(&s.tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&s.tma_bar, 1);
+        mbar_init(&s.mma_bar, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    // constant operand for the row sums: E2M1 1.0 (code 2) with E4M3 scale 1.0
+    for (int i = tid; i < 16 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.ones)[i] = 0x22222222u;
+    for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s.tmem_slot;
+
+    if (!attn_body<D>(s, &tm_q, &tm_k, &tm_v, p, t, bh, tbase) && tid == 0) sa_raise(SA_ERR_TIMEOUT);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+}  // namespace sa

@@ -1,0 +1,324 @@
+// decode.cuh -- one query token per sequence over an NVFP4 KV cache.
+//
+// "Search Your Block Floating Point Scales!" (gist.science summary),
+// "ScaleSearchAttention": the KV cache is kept in 4-bit NVFP4 and attention
+// runs on FP4 tensor cores.  Grouped-query heads: query head h reads kv head
+// h / G, G = Hq / Hkv.
+//
+// One CTA per (b, kv head, split of 4096 keys).  The G query heads of the
+// group form the N side of a swapped MMA so the 128 keys of a tile fill the
+// M = 128 side:
+//   S^T[128 keys, 8] = K_tile (A, TMA, scale atoms) x q^T (B, G rows + zero rows)
+//   per head (column): running max over keys (shuffles + shared memory),
+//   P~ = exp2(S c - m), per 16 keys (16 lanes) scale E4M3(max p/6), E2M1 codes
+//   -> P^T (B operand: 8 rows x 128 keys, 64-byte swizzle) + scale atom
+//   O^T[D, 8] += V^T_tile (A) x P^T,  L[128, 8] += ones(A) x P^T
+// q is quantised in the kernel with the tensor-wide g from a preceding amax
+// pass (same block rule as the pre-pass: 16 channels, max-scaling).
+// Each split writes (m, l, O) unnormalised; decode_combine_kernel merges the
+// splits exactly: O = sum_s 2^(m_s-M) O_s / sum_s 2^(m_s-M) l_s.
+#pragma once
+
+#include "attn.cuh"
+#include "quant.cuh"
+
+namespace sa {
+
+constexpr int kSplit = 4096;
+constexpr int kDecN = 8;  // MMA N (query heads of a group, zero-padded)
+
+template <int D>
+struct DecSmem {
+    uint8_t k[128 * D / 2];    // K tile (A), D/2-byte swizzle
+    uint8_t v[128 * 64];       // V^T tile (A): 128 rows (channels >= D zero-filled), 64-byte swizzle
+    uint8_t ones[128 * 64];    // constant A operand: E2M1 1.0
+    uint8_t q[kDecN * D / 2];  // q^T (B): 8 rows, D/2-byte swizzle
+    uint8_t p[kDecN * 64];     // P^T (B): 8 rows x 128 keys, 64-byte swizzle
+    uint8_t ksf[D / 64 * 512];
+    uint8_t vsf[2 * 512];
+    uint8_t qsf[D / 64 * 512];
+    uint8_t psf[2 * 512];
+    uint8_t onesf[512];
+    float red[4][kDecN];
+    float mnew[kDecN];
+    float alpha[kDecN];
+    uint64_t tma_bar;
+    uint64_t mma_bar;
+    uint32_t tmem_slot;
+};
+
+// TMEM columns (64 allocated)
+constexpr uint32_t DM_S = 0, DM_O = 8, DM_L = 16, DM_SFK = 24, DM_SFQ = 32, DM_SFV = 40, DM_SFP = 48, DM_SF1 = 56;
+
+struct DecParams {
+    const uint16_t* q;  // bf16 [B, Hq, D]
+    const unsigned* q_amax;
+    const uint8_t* k_sf;
+    const uint8_t* v_sf;
+    const float* k_g;
+    const float* v_g;
+    float* part;  // [B*Hq, nsplit, D + 2]: O (D), l, m
+    int L, Hq, Hkv, G, nsplit, RTk, CKv;
+    float sm_scale;
+};
+
+template <int D>
+SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMap* tm_v, const DecParams& p,
+                        int b, int hk, int split, uint32_t tbase)
+{
+    constexpr int KB = D / 64;
+    constexpr uint32_t KSW = D == 128 ? 4u : 6u;
+    constexpr uint32_t KSBO = 8 * D / 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int bhk = b * p.Hkv + hk;
+
+    // ---- quantise the group's query rows (q^T operand + its scale atom)
+    {
+        float g, inv_g;
+        tensor_scale(__uint_as_float(*p.q_amax), g, inv_g);
+        for (int e = tid; e < kDecN * D / 2; e += blockDim.x) s.q[e] = 0;
+        for (int e = tid; e < KB * 512; e += blockDim.x) s.qsf[e] = 0;
+        __syncthreads();
+        const int nblk = p.G * (D / 16);
+        if (tid < nblk) {
+            const int hi = tid / (D / 16), j = tid % (D / 16);
+            const uint16_t* src = p.q + ((size_t)b * p.Hq + hk * p.G + hi) * D + j * 16;
+            float xt[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) xt[i] = __fmul_rn(bf16_bits_to_f32(src[i]), inv_g);
+            uint32_t c0, c1, sc;
+            int off;
+            quant16<false>(xt, 0, 1, c0, c1, sc, off);
+            // row hi, bytes 8j..8j+7 of a (D/2)-byte row, swizzled in 16-byte chunks
+            const int byte = 8 * j;
+            const int chunk = byte >> 4;
+            const int sw = D == 128 ? (chunk ^ ((hi & 7) >> 1)) : (chunk ^ ((hi & 7) >> 2));
+            *reinterpret_cast<uint2*>(s.q + hi * (D / 2) + sw * 16 + (byte & 15)) = make_uint2(c0, c1);
+            s.qsf[(j >> 2) * 512 + sf_atom_offset((uint32_t)hi, (uint32_t)(j & 3))] = (uint8_t)sc;
+        }
+    }
+    float gq, inv_gq;
+    tensor_scale(__uint_as_float(*p.q_amax), gq, inv_gq);
+    const float cexp = gq * p.k_g[0] * p.sm_scale * kLog2e;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    uint32_t tma_phase = 0, mma_phase = 0;
+    if (tid == 0) {
+        tc_fence_after();
+        for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
+        tc_cp_sf(tbase + DM_SF1, smem_u32(s.onesf));
+    }
+
+    float m2[kDecN];
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) m2[h] = -INFINITY;
+    const int key0 = split * kSplit;
+    const int nkeys = min(kSplit, p.L - key0);
+    const int ntiles = nkeys / 128;
+    for (int u = 0; u < ntiles; u++) {
+        const int ktile = key0 / 128 + u;
+        if (tid == 0) {
+            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + 128 * 64 + 2 * 512);
+            tma_load_3d(s.k, tm_k, &s.tma_bar, 0, ktile * 128, bhk);
+            bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + ktile) * KB * 512, KB * 512, &s.tma_bar);
+            tma_load_3d(s.v, tm_v, &s.tma_bar, ktile * 64, 0, bhk);
+            bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * ktile) * 512, 2 * 512, &s.tma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
+        tma_phase ^= 1;
+        if (tid == 0) {
+            tc_fence_after();
+            for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFK + 4 * kb, smem_u32(s.ksf + 512 * kb));
+            for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFV + 4 * kb, smem_u32(s.vsf + 512 * kb));
+            for (int kb = 0; kb < KB; kb++)
+                mma_fp4(tbase + DM_S, make_sdesc(smem_u32(s.k) + 32 * kb, KSBO, 16, KSW),
+                        make_sdesc(smem_u32(s.q) + 32 * kb, KSBO, 16, KSW), idesc_fp4(128, kDecN),
+                        tbase + DM_SFK + 4 * kb, tbase + DM_SFQ + 4 * kb, kb > 0);
+            tc_commit(&s.mma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // ---- scores of this thread's key for the 8 columns
+        float sv[kDecN];
+        {
+            uint32_t r[kDecN];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+                "tcgen05.wait::ld.sync.aligned;"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                : "r"(tbase + lane_off + DM_S)
+                : "memory");
+#pragma unroll
+            for (int h = 0; h < kDecN; h++) sv[h] = __uint_as_float(r[h]);
+        }
+        // column max over the 128 keys
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) {
+            float mx = sv[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) s.red[warp][h] = mx;
+        }
+        __syncthreads();
+        if (tid < kDecN) {
+            const float tmax = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
+            const float mo = m2[tid];
+            const float mn = fmaxf(mo, tmax * cexp);
+            s.mnew[tid] = mn;
+            s.alpha[tid] = ex2f(mo - mn);
+        }
+        __syncthreads();
+        float alpha[kDecN];
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) {
+            m2[h] = s.mnew[h];
+            alpha[h] = s.alpha[h];
+        }
+        // P^T codes and scales: block of 16 keys = 16 lanes
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) {
+            const float x = fmaf(sv[h], cexp, kLog2_2688 - m2[h]);
+            float bm = x;
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const uint32_t sc = f32_to_e4m3(ex2f(bm) * (1.0f / 6.0f));
+            const float y = sc ? ex2f(x - lg2f(e4m3_to_f32(sc))) : 0.0f;
+            const uint32_t code = pack8_e2m1(y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 15u;
+            const uint32_t hi_code = __shfl_down_sync(0xffffffffu, code, 1);
+            if ((lane & 1) == 0) {
+                const int byte = tid >> 1;        // key pair index within the 128 keys
+                const int chunk = byte >> 4;
+                const int sw = chunk ^ ((h & 7) >> 1);
+                s.p[h * 64 + sw * 16 + (byte & 15)] = (uint8_t)(code | (hi_code << 4));
+            }
+            if ((lane & 15) == 0) {
+                const int blk = tid >> 4;  // 0..7 over the 128 keys
+                s.psf[(blk >> 2) * 512 + sf_atom_offset((uint32_t)h, (uint32_t)(blk & 3))] = (uint8_t)sc;
+            }
+        }
+        // rescale O^T and L columns whose head max moved
+        bool any = false;
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) any |= alpha[h] != 1.0f;
+        if (u > 0 && any) {
+            uint32_t r[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+                "%14, %15}, [%16];\n\t"
+                "tcgen05.wait::ld.sync.aligned;"
+                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                  "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                  "=r"(r[15])
+                : "r"(tbase + lane_off + DM_O)
+                : "memory");
+#pragma unroll
+            for (int i = 0; i < 16; i++) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha[i & 7]);
+            asm volatile(
+                "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+                "%13, %14, %15, %16};\n\t"
+                "tcgen05.wait::st.sync.aligned;" ::"r"(tbase + lane_off + DM_O),
+                "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+                "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+                : "memory");
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
+            for (int kb = 0; kb < 2; kb++) {
+                const uint64_t pd = make_sdesc(smem_u32(s.p) + 32 * kb, 512, 16, 4);
+                const uint32_t acc = (u > 0 || kb > 0) ? 1u : 0u;
+                mma_fp4(tbase + DM_O, make_sdesc(smem_u32(s.v) + 32 * kb, 512, 16, 4), pd, idesc_fp4(128, kDecN),
+                        tbase + DM_SFV + 4 * kb, tbase + DM_SFP + 4 * kb, acc);
+                mma_fp4(tbase + DM_L, make_sdesc(smem_u32(s.ones) + 32 * kb, 512, 16, 4), pd,
+                        idesc_fp4(128, kDecN), tbase + DM_SF1, tbase + DM_SFP + 4 * kb, acc);
+            }
+            tc_commit(&s.mma_bar);
+        }
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        mma_phase ^= 1;
+        tc_fence_after();
+    }
+
+    // ---- write this split's unnormalised O (lane = channel), l and m
+    uint32_t o[kDecN], l[kDecN];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%9, %10, %11, %12, %13, %14, %15, %16}, [%17];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]),
+          "=r"(l[0]), "=r"(l[1]), "=r"(l[2]), "=r"(l[3]), "=r"(l[4]), "=r"(l[5]), "=r"(l[6]), "=r"(l[7])
+        : "r"(tbase + lane_off + DM_O), "r"(tbase + lane_off + DM_L)
+        : "memory");
+    for (int h = 0; h < p.G; h++) {
+        float* dst = p.part + (((size_t)b * p.Hq + hk * p.G + h) * p.nsplit + split) * (D + 2);
+        if (tid < D) dst[tid] = __uint_as_float(o[h]);
+        if (tid == 0) {
+            dst[D] = __uint_as_float(l[h]);
+            dst[D + 1] = m2[h];
+        }
+    }
+    return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                     const __grid_constant__ CUtensorMap tm_v, const DecParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    DecSmem<D>& s = *reinterpret_cast<DecSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                   ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    if (warp == 0) {
+        tmem_alloc(&s.tmem_slot, 64);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(&s.tma_bar, 1);
+        mbar_init(&s.mma_bar, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    for (int i = tid; i < 128 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.ones)[i] = 0x22222222u;
+    for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
+    for (int i = tid; i < kDecN * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.p)[i] = 0u;
+    for (int i = tid; i < 2 * 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.psf)[i] = 0u;
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = s.tmem_slot;
+    if (!decode_body<D>(s, &tm_k, &tm_v, p, b, hk, split, tbase) && tid == 0) sa_raise(SA_ERR_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 64);
+}
+
+// Merge the splits of one (b, query head): thread per channel.
+__global__ void decode_combine_kernel(const float* __restrict__ part, int nsplit, int D, const float* __restrict__ v_g,
+                                      float* __restrict__ out)
+{
+    const size_t bq = blockIdx.x;
+    const int d = threadIdx.x;
+    const float* pp = part + bq * nsplit * (D + 2);
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; s++) M = fmaxf(M, pp[s * (D + 2) + D + 1]);
+    float num = 0.0f, den = 0.0f;
+    for (int s = 0; s < nsplit; s++) {
+        const float w = ex2f(pp[s * (D + 2) + D + 1] - M);
+        den = fmaf(w, pp[s * (D + 2) + D], den);
+        if (d < D) num = fmaf(w, pp[s * (D + 2) + d], num);
+    }
+    if (d < D) out[bq * D + d] = num / den * v_g[0];
+}
+
+}  // namespace sa

@@ -1,0 +1,361 @@
+// sa.cu -- the C ABI of libsa (declared in include/sa.h): argument checks,
+// TMA tensor maps, workspace carving and kernel launches.  One translation
+// unit so the device status word is a single object.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "decode.cuh"
+#include "quant.cuh"
+#include "select.cuh"
+
+using namespace sa;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D byte tensor {d0 (contiguous), d1, d2}; box {b0, b1, 1}.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                 uint32_t b1, CUtensorMapSwizzle swz)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0, d0 * d1};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int rt_ck(int R, int C, int* RT, int* CK)
+{
+    *RT = sa_cdiv(R, 128);
+    *CK = sa_cdiv(C, 64);
+    return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_status_string(sa_status s)
+{
+    switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    case SA_ERR_NONFINITE: return "SA_ERR_NONFINITE";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    case SA_ERR_DEVICE_ASSERT: return "SA_ERR_DEVICE_ASSERT";
+    }
+    return "SA_ERR_UNKNOWN";
+}
+
+sa_status sa_device_status(cudaStream_t stream, int reset)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_sa_status, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+    if (reset) {
+        int z = 0;
+        if (cudaMemcpyToSymbol(g_sa_status, &z, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+    }
+    return (sa_status)v;
+}
+
+size_t sa_codes_bytes(int B, int H, int N, int D, sa_role role)
+{
+    (void)role;
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    return (size_t)B * H * N * D / 2;
+}
+
+size_t sa_scales_bytes(int B, int H, int N, int D, sa_role role)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    int RT, CK;
+    if (role == SA_ROLE_V)
+        rt_ck(D, N, &RT, &CK);
+    else
+        rt_ck(N, D, &RT, &CK);
+    return (size_t)B * H * RT * CK * 512;
+}
+
+size_t sa_quant_workspace_size(int B, int H, int N, int D, sa_role role)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    return quant_ws_layout(nullptr, B, H, N, D, role).bytes;
+}
+
+sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role role, int smooth,
+                         sa_scale_mode mode, int f_lo, int f_hi, uint8_t* codes_dev, uint8_t* scales_dev,
+                         float* g_dev, float* k_mean_dev, int8_t* ss_off_dev, void* ws_dev, size_t ws_bytes,
+                         cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+    if (role != SA_ROLE_Q && role != SA_ROLE_K && role != SA_ROLE_V) return SA_ERR_INVALID_ARG;
+    if (mode != SA_SCALE_MAX && mode != SA_SCALE_SEARCH) return SA_ERR_INVALID_ARG;
+    if (mode == SA_SCALE_SEARCH && !(f_lo >= -16 && f_lo <= 0 && f_hi > 0 && f_hi <= 16)) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if (N % 16) return SA_ERR_INVALID_ARG;
+    if ((size_t)B * H * N == 0) return SA_OK;
+    if (!x_dev || !codes_dev || !scales_dev || !g_dev || !ws_dev) return SA_ERR_INVALID_ARG;
+    if (!aligned16(x_dev) || ((uintptr_t)codes_dev & 7u) || ((uintptr_t)ws_dev & 255u)) return SA_ERR_INVALID_ARG;
+    if (role != SA_ROLE_K) smooth = 0;
+    QuantWs w = quant_ws_layout(ws_dev, B, H, N, D, role);
+    if (ws_bytes < w.bytes) return SA_ERR_WORKSPACE;
+    const size_t BH = (size_t)B * H;
+    const int T = sa_cdiv(N, kTile);
+
+    // padding bytes of the scale atoms must read as zero
+    const bool pad = role == SA_ROLE_V ? (D % 128 != 0 || N % 64 != 0) : (N % 128 != 0);
+    if (pad && cudaMemsetAsync(scales_dev, 0, sa_scales_bytes(B, H, N, D, role), stream) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (cudaMemsetAsync(w.amax, 0, 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+
+    float* kmean = k_mean_dev ? k_mean_dev : w.kmean;
+    if (smooth) {
+        dim3 g1(sa_cdiv(T, 256 / (D / 2)), (unsigned)BH);
+        if (D == 128)
+            kstats_kernel<128><<<g1, 256, 0, stream>>>((const uint32_t*)x_dev, N, T, w.psum, w.pmax, w.pmin);
+        else
+            kstats_kernel<64><<<g1, 256, 0, stream>>>((const uint32_t*)x_dev, N, T, w.psum, w.pmax, w.pmin);
+        SA_CHECK_LAUNCH();
+        kfinal_kernel<<<(unsigned)BH, 128, 0, stream>>>(w.psum, w.pmax, w.pmin, N, T, D, kmean, w.amax);
+        SA_CHECK_LAUNCH();
+    } else {
+        size_t n16 = BH * N * D / 8;
+        amax_bf16_kernel<<<grid_for(n16, 256 * 4), 256, 0, stream>>>((const uint4*)x_dev, n16, w.amax);
+        SA_CHECK_LAUNCH();
+    }
+
+    const bool ss = mode == SA_SCALE_SEARCH;
+    if (role == SA_ROLE_V) {
+        size_t nblk = BH * (N / 16) * D;
+        int grid = grid_for(nblk, 256);
+        if (ss)
+            quant_v_kernel<true><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk, N, D, w.amax, f_lo, f_hi,
+                                                           codes_dev, scales_dev, ss_off_dev, g_dev);
+        else
+            quant_v_kernel<false><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk, N, D, w.amax, f_lo, f_hi,
+                                                            codes_dev, scales_dev, ss_off_dev, g_dev);
+    } else {
+        size_t nblk = BH * N * (D / 16);
+        int grid = grid_for(nblk, 256);
+        const uint4* x = (const uint4*)x_dev;
+        uint2* c = (uint2*)codes_dev;
+#define SA_QR(DD, SM, SS)                                                                                    \
+    quant_rows_kernel<DD, SM, SS><<<grid, 256, 0, stream>>>(x, nblk, N, T, kmean, w.amax, f_lo, f_hi, c, \
+                                                           scales_dev, ss_off_dev, g_dev)
+        if (D == 128) {
+            if (smooth) {
+                if (ss) SA_QR(128, true, true); else SA_QR(128, true, false);
+            } else {
+                if (ss) SA_QR(128, false, true); else SA_QR(128, false, false);
+            }
+        } else {
+            if (smooth) {
+                if (ss) SA_QR(64, true, true); else SA_QR(64, true, false);
+            } else {
+                if (ss) SA_QR(64, false, true); else SA_QR(64, false, false);
+            }
+        }
+#undef SA_QR
+    }
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+size_t sa_select_workspace_size(int B, int H, int N, int D)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    return select_ws_bytes(B, H, N, D);
+}
+
+sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, int N, int D, int causal,
+                           int frac_bp, uint8_t* mask_dev, int32_t* nsel_dev, void* ws_dev, size_t ws_bytes,
+                           cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || N < 0 || frac_bp < 0 || frac_bp > 10000) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if ((size_t)B * H * N == 0) return SA_OK;
+    if (!q_dev || !k_dev || !mask_dev || !ws_dev) return SA_ERR_INVALID_ARG;
+    if ((uintptr_t)ws_dev & 255u) return SA_ERR_INVALID_ARG;
+    if (ws_bytes < select_ws_bytes(B, H, N, D)) return SA_ERR_WORKSPACE;
+    const int T = sa_cdiv(N, 128);
+    const size_t BH = (size_t)B * H;
+    float* qbar = (float*)ws_dev;
+    float* kbar = (float*)((char*)ws_dev + sa_align256(BH * T * D * sizeof(float)));
+    float* scores = (float*)((char*)ws_dev + 2 * sa_align256(BH * T * D * sizeof(float)));
+    pool_kernel<<<dim3(T, (unsigned)BH, 2), 128, 0, stream>>>((const uint16_t*)q_dev, (const uint16_t*)k_dev, N, D, T,
+                                                             qbar, kbar);
+    SA_CHECK_LAUNCH();
+    score_kernel<<<dim3(sa_cdiv(T, 32), sa_cdiv(T, 8), (unsigned)BH), 256, 0, stream>>>(qbar, kbar, D, T, scores);
+    SA_CHECK_LAUNCH();
+    topk_kernel<<<(unsigned)BH, kTopkThreads, 0, stream>>>(scores, T, causal, frac_bp, mask_dev, nsel_dev);
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,
+                      const uint8_t* k_codes_dev, const uint8_t* k_scales_dev, const float* k_g_dev,
+                      const uint8_t* v_codes_dev, const uint8_t* v_scales_dev, const float* v_g_dev, int B, int H,
+                      int N, int D, int causal, float sm_scale, const uint8_t* mask_dev, const void* q_bf16_dev,
+                      const void* k_bf16_dev, const void* v_bf16_dev, const float* k_mean_dev, float* out_dev,
+                      float* lse_dev, cudaStream_t stream)
+{
+    (void)q_bf16_dev;
+    (void)k_bf16_dev;
+    (void)v_bf16_dev;
+    (void)k_mean_dev;
+    if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if (N % 32) return SA_ERR_INVALID_ARG;
+    if ((size_t)B * H * N == 0) return SA_OK;
+    if (!q_codes_dev || !q_scales_dev || !q_g_dev || !k_codes_dev || !k_scales_dev || !k_g_dev || !v_codes_dev ||
+        !v_scales_dev || !v_g_dev || !out_dev)
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q_codes_dev) || !aligned16(k_codes_dev) || !aligned16(v_codes_dev) || !aligned16(q_scales_dev) ||
+        !aligned16(k_scales_dev) || !aligned16(v_scales_dev) || !aligned16(out_dev))
+        return SA_ERR_INVALID_ARG;
+    if (mask_dev) return SA_ERR_UNSUPPORTED;
+    if (!(sm_scale > 0.0f)) sm_scale = 1.0f / sqrtf((float)D);
+    const uint64_t BH = (uint64_t)B * H;
+    const CUtensorMapSwizzle qsw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUtensorMap tq, tk, tv;
+    if (!make_map_u8(&tq, q_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
+        !make_map_u8(&tk, k_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
+        !make_map_u8(&tv, v_codes_dev, N / 2, D, BH, 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
+        return SA_ERR_CUDA;
+    AttnParams p{};
+    p.q_sf = q_scales_dev;
+    p.k_sf = k_scales_dev;
+    p.v_sf = v_scales_dev;
+    p.q_g = q_g_dev;
+    p.k_g = k_g_dev;
+    p.v_g = v_g_dev;
+    p.out = out_dev;
+    p.lse = lse_dev;
+    p.N = N;
+    p.H = H;
+    p.T = sa_cdiv(N, 128);
+    p.CKv = sa_cdiv(N, 64);
+    p.causal = causal ? 1 : 0;
+    p.sm_scale = sm_scale;
+    dim3 grid(p.T, H, B);
+    // one CTA per SM (the CTA owns all 512 TMEM columns)
+    const int smem = 116 * 1024;
+    if (D == 128) {
+        static_assert(sizeof(AttnSmem<128>) + 1024 <= 116 * 1024, "smem");
+        if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        attn_fwd_kernel<128><<<grid, 128, smem, stream>>>(tq, tk, tv, p);
+    } else {
+        if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        attn_fwd_kernel<64><<<grid, 128, smem, stream>>>(tq, tk, tv, p);
+    }
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+size_t sa_decode_workspace_size(int B, int Hq, int Hkv, int L, int D)
+{
+    if (B < 0 || Hq < 0 || Hkv <= 0 || L < 0 || D < 0) return 0;
+    const int nsplit = sa_cdiv(L, kSplit);
+    return 256 + sa_align256((size_t)B * Hq * nsplit * (D + 2) * sizeof(float));
+}
+
+sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                               const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
+                               const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
+                               float* out_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream)
+{
+    if (B < 0 || Hq < 0 || Hkv <= 0 || L < 0) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if (Hq % Hkv || Hq / Hkv > kDecN || L % 128) return SA_ERR_INVALID_ARG;
+    if ((size_t)B * Hq == 0) return SA_OK;
+    if (L == 0) return SA_ERR_INVALID_ARG;
+    if (!q_dev || !k_codes_dev || !k_scales_dev || !k_g_dev || !v_codes_dev || !v_scales_dev || !v_g_dev ||
+        !out_dev || !ws_dev)
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q_dev) || !aligned16(k_codes_dev) || !aligned16(v_codes_dev) || !aligned16(k_scales_dev) ||
+        !aligned16(v_scales_dev) || ((uintptr_t)ws_dev & 255u))
+        return SA_ERR_INVALID_ARG;
+    if (ws_bytes < sa_decode_workspace_size(B, Hq, Hkv, L, D)) return SA_ERR_WORKSPACE;
+    if (!(sm_scale > 0.0f)) sm_scale = 1.0f / sqrtf((float)D);
+    const uint64_t BHk = (uint64_t)B * Hkv;
+    const int nsplit = sa_cdiv(L, kSplit);
+    unsigned* amax = (unsigned*)ws_dev;
+    float* part = (float*)((char*)ws_dev + 256);
+    if (cudaMemsetAsync(amax, 0, 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+    size_t n16 = (size_t)B * Hq * D / 8;
+    amax_bf16_kernel<<<grid_for(n16, 256), 256, 0, stream>>>((const uint4*)q_dev, n16, amax);
+    SA_CHECK_LAUNCH();
+    const CUtensorMapSwizzle ksw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUtensorMap tk, tv;
+    if (!make_map_u8(&tk, k_codes_dev, D / 2, L, BHk, D / 2, 128, ksw) ||
+        !make_map_u8(&tv, v_codes_dev, L / 2, D, BHk, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+        return SA_ERR_CUDA;
+    DecParams p{};
+    p.q = (const uint16_t*)q_dev;
+    p.q_amax = amax;
+    p.k_sf = k_scales_dev;
+    p.v_sf = v_scales_dev;
+    p.k_g = k_g_dev;
+    p.v_g = v_g_dev;
+    p.part = part;
+    p.L = L;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.nsplit = nsplit;
+    p.RTk = sa_cdiv(L, 128);
+    p.CKv = sa_cdiv(L, 64);
+    p.sm_scale = sm_scale;
+    dim3 grid(nsplit, Hkv, B);
+    if (D == 128) {
+        const int smem = (int)sizeof(DecSmem<128>) + 1024;
+        if (cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        decode_kernel<128><<<grid, 128, smem, stream>>>(tk, tv, p);
+    } else {
+        const int smem = (int)sizeof(DecSmem<64>) + 1024;
+        if (cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return SA_ERR_CUDA;
+        decode_kernel<64><<<grid, 128, smem, stream>>>(tk, tv, p);
+    }
+    SA_CHECK_LAUNCH();
+    decode_combine_kernel<<<(unsigned)(B * Hq), 128, 0, stream>>>(part, nsplit, D, v_g_dev, out_dev);
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+"""C-ABI checks that need no GPU: libsa.so builds, loads, exports every
+function that include/sa.h declares, sizes its buffers as documented, and
+rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_quantized_attention_channel_b200 as sa
+from bit_quantized_attention_channel_b200 import build as sabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    sabuild.build()
+    return sa.lib()
+
+
+def declared_functions():
+    hdr = open(os.path.join(ROOT, "include", "sa.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", hdr)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for i, name in enumerate(sa.STATUS):
+        assert L.sa_status_string(i).decode() == name
+
+
+def test_buffer_sizes(L):
+    # Q/K: codes B*H*N*D/2; scales: 512-byte atoms per (128 rows, 64 columns)
+    assert L.sa_codes_bytes(2, 16, 4096, 128, 0) == 2 * 16 * 4096 * 64
+    assert L.sa_scales_bytes(2, 16, 4096, 128, 0) == 2 * 16 * 32 * 2 * 512
+    # ragged N rounds the row tiles up
+    assert L.sa_scales_bytes(1, 1, 400, 64, 1) == 4 * 1 * 512
+    # V: rows are channels (one 128-row tile for D <= 128), chunks along tokens
+    assert L.sa_scales_bytes(1, 2, 4096, 128, 2) == 2 * 1 * 64 * 512
+    assert L.sa_scales_bytes(1, 1, 400, 64, 2) == 1 * 1 * 7 * 512
+    assert L.sa_quant_workspace_size(1, 1, 256, 64, 0) == 256
+    assert L.sa_quant_workspace_size(1, 1, 256, 64, 1) > 256
+
+
+def test_rejects_bad_arguments_before_launch(L):
+    n = None
+    # unsupported head dim
+    assert L.sa_quant_nvfp4(n, 1, 1, 128, 96, 0, 0, 0, -2, 6, n, n, n, n, n, n, 0, n) == 2
+    # N not a multiple of 16
+    assert L.sa_quant_nvfp4(n, 1, 1, 100, 64, 0, 0, 0, -2, 6, n, n, n, n, n, n, 0, n) == 1
+    # bad ScaleSearch range
+    assert L.sa_quant_nvfp4(n, 1, 1, 128, 64, 0, 0, 1, 1, 6, n, n, n, n, n, n, 0, n) == 1
+    # empty tensor: valid, nothing launched
+    assert L.sa_quant_nvfp4(n, 0, 1, 128, 64, 0, 0, 0, -2, 6, n, n, n, n, n, n, 0, n) == 0
+    # null buffers
+    assert L.sa_quant_nvfp4(n, 1, 1, 128, 64, 0, 0, 0, -2, 6, n, n, n, n, n, n, 0, n) == 1
+    # attention: N % 32, unsupported D, null pointers
+    assert L.sa_attn_fwd(*([n] * 9), 1, 1, 48, 64, 0, 0.0, *([n] * 8)) == 1
+    assert L.sa_attn_fwd(*([n] * 9), 1, 1, 64, 80, 0, 0.0, *([n] * 8)) == 2
+    assert L.sa_attn_fwd(*([n] * 9), 1, 1, 64, 64, 0, 0.0, *([n] * 8)) == 1
+    # decode: Hq % Hkv, L % 128
+    assert L.sa_attn_decode_kvfp4(*([n] * 7), 1, 6, 4, 256, 128, 0.0, n, n, 0, n) == 1
+    assert L.sa_attn_decode_kvfp4(*([n] * 7), 1, 8, 2, 200, 128, 0.0, n, n, 0, n) == 1
+    # selector: budget out of range
+    assert L.sa_thrift_select(n, n, 1, 1, 256, 64, 1, 20000, n, n, n, 0, n) == 1
+
+
+def test_scales_to_logical_roundtrip():
+    import numpy as np
+    import torch
+
+    B, H, N, D = 1, 2, 400, 64
+    R, C = N, D
+    logical = torch.randint(0, 127, (B, H, R, C // 16), dtype=torch.uint8)
+    RT, CK = (R + 127) // 128, (C + 63) // 64
+    atoms = torch.zeros(B * H * RT * CK * 512, dtype=torch.uint8)
+    for bh in range(B * H):
+        for r in range(R):
+            for j in range(C // 16):
+                a = (bh * RT + r // 128) * CK + j // 4
+                atoms[a * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4] = logical.view(B * H, R, -1)[bh, r, j]
+    back = sa.scales_to_logical(atoms, B, H, N, D, "q")
+    assert torch.equal(back, logical)

@@ -1,0 +1,264 @@
+"""GPU path (through the C ABI) vs the CPU oracle on the same seeded inputs.
+
+Bar (from the method's definition of what is exact):
+  * bit-exact: E2M1 codes, E4M3 scales, per-tensor g, K channel means,
+    ScaleSearch offsets, selector masks and counts;
+  * attention / decode outputs: max |O_gpu - O_oracle| <= 2e-3 * max |O_oracle|
+    and cosine >= 0.9999 (P is requantised from FP32 scores on the GPU and
+    from FP64 scores in the oracle, so individual P codes may differ where a
+    score sits on a rounding boundary; the output tolerance covers that).
+The oracle always quantises the raw inputs itself; nothing it consumes comes
+from the GPU.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_attention_channel_b200 as sa
+import oracle as orc
+from bit_quantized_attention_channel_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ATOL_REL = 2e-3
+COS_MIN = 0.9999
+
+
+# ------------------------------------------------------------------ helpers
+def status_ok():
+    st = sa.sa_device_status(reset=True)
+    assert st == 0, sa.STATUS[st]
+
+
+def gpu_quant(x_cpu, role, smooth=True, mode="max"):
+    r = sa.sa_quant_nvfp4(x_cpu.cuda(), role, smooth=smooth, mode=mode, ss_offsets=True)
+    status_ok()
+    return r
+
+
+def assert_quant_equal(rg, ro, tag=""):
+    B, H, N, D = rg.shape
+    codes = rg.codes.cpu().numpy().reshape(ro.codes.shape)
+    bad = codes != ro.codes
+    assert not bad.any(), f"{tag}: {bad.sum()} code bytes differ, first at {np.argwhere(bad)[:3].tolist()}: " \
+                          f"gpu {codes[bad][:8]} oracle {ro.codes[bad][:8]}"
+    sc = sa.scales_to_logical(rg.scales.cpu(), B, H, N, D, rg.role).numpy()
+    bad = sc != ro.scales
+    assert not bad.any(), f"{tag}: {bad.sum()} scales differ: gpu {sc[bad][:8]} oracle {ro.scales[bad][:8]}"
+    g = rg.g.cpu().numpy()
+    assert g[0] == np.float32(ro.g) and g[1] == np.float32(ro.inv_g), (tag, g, ro.g, ro.inv_g)
+    if ro.k_mean is not None:
+        assert np.array_equal(rg.k_mean.cpu().numpy(), ro.k_mean), tag
+    off = rg.ss_off.cpu().numpy()[: ro.ss_off.size].reshape(ro.ss_off.shape)
+    assert np.array_equal(off, ro.ss_off), f"{tag}: {np.sum(off != ro.ss_off)} ScaleSearch offsets differ"
+    # padding of the scale atoms is zero
+    total = int(rg.scales.numel())
+    R, C = (D, N) if rg.role == "v" else (N, D)
+    if total > B * H * R * (C // 16):
+        logical_sum = int(sc.astype(np.int64).sum())
+        assert int(rg.scales.cpu().numpy().astype(np.int64).sum()) == logical_sum, f"{tag}: padding not zero"
+
+
+def check_close(got, ref, tag=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = float(np.max(np.abs(got - ref)))
+    scale = float(np.max(np.abs(ref)))
+    cos = float(np.sum(got * ref) / (np.linalg.norm(got) * np.linalg.norm(ref)))
+    print(f"{tag}: max|d|/max|O| = {err / scale:.2e}  cos = {cos:.7f}")
+    assert err <= ATOL_REL * scale, (tag, err, scale)
+    assert cos >= COS_MIN, (tag, cos)
+
+
+def exact_rows(q, k, v, causal, rows, sm):
+    """FP64 exact softmax attention on raw bf16 inputs for selected rows."""
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    B, H, N, D = qd.shape
+    out = np.zeros((B, H, len(rows), D))
+    for i, r in enumerate(rows):
+        s = np.einsum("bhd,bhjd->bhj", qd[:, :, r], kd) * sm
+        if causal:
+            s[:, :, r + 1:] = -np.inf
+        s -= s.max(-1, keepdims=True)
+        p = np.exp(s)
+        out[:, :, i] = np.einsum("bhj,bhjd->bhd", p, vd) / p.sum(-1)[..., None]
+    return out
+
+
+def quality(got, ref):
+    cos = float(np.sum(got * ref) / (np.linalg.norm(got) * np.linalg.norm(ref)))
+    rl1 = float(np.abs(got - ref).sum() / np.abs(ref).sum())
+    return cos, rl1
+
+
+def sample_rows(N):
+    T = (N + 127) // 128
+    rows = set()
+    for t in sorted({0, 1, T // 2, T - 2, T - 1}):
+        if t < 0:
+            continue
+        for o in (0, 1, 63, 64, 127):
+            r = t * 128 + o
+            if r < N:
+                rows.add(r)
+    return np.array(sorted(rows), np.int32)
+
+
+# ------------------------------------------------------------------ inputs
+_cache = {}
+
+
+def inputs(name, **shape):
+    key = (name, tuple(sorted(shape.items())))
+    if key not in _cache:
+        _cache[key] = wl.prefill_inputs(name, **shape)
+    return _cache[key]
+
+
+# ------------------------------------------------------------------ quant
+QUANT_CASES = [
+    ("tiny", {}, "max"),
+    ("tiny", {"N": 400}, "search"),         # ragged: N not a multiple of 128 or 64
+    ("llm", {}, "max"),
+    ("llm", {}, "search"),
+    ("video", {"H": 2}, "search"),
+    ("longctx", {"H": 2, "N": 8192}, "max"),
+]
+
+
+@pytest.mark.parametrize("name,shape,mode", QUANT_CASES)
+def test_quant_bit_exact(name, shape, mode):
+    q, k, v = inputs(name, **shape)
+    for role, x in (("q", q), ("k", k), ("v", v)):
+        rg = gpu_quant(x, role, smooth=True, mode=mode)
+        ro = orc.quantize(x, role, smooth=True, search=mode == "search")
+        assert_quant_equal(rg, ro, f"{name}{shape}/{role}/{mode}")
+
+
+def test_quant_k_unsmoothed_and_zero_tensor():
+    _, k, _ = inputs("tiny")
+    assert_quant_equal(gpu_quant(k, "k", smooth=False), orc.quantize(k, "k", smooth=False), "k unsmoothed")
+    z = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    for role in ("q", "k", "v"):
+        assert_quant_equal(gpu_quant(z, role, mode="search"), orc.quantize(z, role, search=True), f"zero/{role}")
+
+
+def test_quant_nonfinite_is_reported():
+    x = torch.randn(1, 1, 128, 64).to(torch.bfloat16)
+    x[0, 0, 5, 7] = float("nan")
+    sa.sa_quant_nvfp4(x.cuda(), "q")
+    assert sa.sa_device_status(reset=True) == 4  # SA_ERR_NONFINITE
+    status_ok()
+
+
+@pytest.mark.parametrize("name", ["video", "longctx"])
+def test_quant_bit_exact_full_size(name):
+    """Full-size pre-pass of the long workloads (every element compared)."""
+    q, k, v = inputs(name)
+    w = wl.WORKLOADS[name]
+    mode = "search" if "search" in w.scale_modes else "max"
+    for role, x in (("q", q), ("k", k), ("v", v)):
+        assert_quant_equal(gpu_quant(x, role, mode=mode), orc.quantize(x, role, search=mode == "search"),
+                           f"{name}/{role}")
+
+
+# ------------------------------------------------------------------ selector
+@pytest.mark.parametrize("causal,frac", [(False, 500), (True, 500), (True, 1000), (False, 0), (True, 10000)])
+def test_select_bit_exact_small(causal, frac):
+    q, k, _ = inputs("longctx", H=3, N=1024 + 256)
+    mg, ng = sa.sa_thrift_select(q.cuda(), k.cuda(), causal, frac)
+    status_ok()
+    mo, no = orc.thrift_select(q, k, causal, frac)
+    assert np.array_equal(ng.cpu().numpy(), no)
+    assert np.array_equal(mg.cpu().numpy(), mo)
+
+
+def test_select_ties_break_to_lower_index():
+    q = torch.ones(1, 1, 1024, 64, dtype=torch.bfloat16)
+    mg, ng = sa.sa_thrift_select(q.cuda(), q.cuda(), True, 1000)
+    status_ok()
+    mo, no = orc.thrift_select(q, q, True, 1000)
+    assert np.array_equal(mg.cpu().numpy(), mo) and np.array_equal(ng.cpu().numpy(), no)
+
+
+def test_select_bit_exact_full_size():
+    """Selector on the full long-context workload (B1 H32 N65536, 5 %)."""
+    q, k, _ = inputs("longctx")
+    mg, ng = sa.sa_thrift_select(q.cuda(), k.cuda(), True, 500)
+    status_ok()
+    mo, no = orc.thrift_select(q, k, True, 500)
+    assert np.array_equal(ng.cpu().numpy(), no)
+    assert (no == 6567).all()
+    assert np.array_equal(mg.cpu().numpy(), mo)
+
+
+# ------------------------------------------------------------------ attention
+ATTN_CASES = [
+    ("tiny", {}, False, "max", None),                  # every row compared
+    ("tiny", {}, True, "max", None),
+    ("tiny", {"N": 416, "D": 128}, True, "max", None),  # ragged last tile (416 = 3*128 + 32)
+    ("tiny", {"N": 352}, False, "search", None),       # ragged, D = 64
+    ("tiny", {"N": 128, "H": 1}, True, "max", None),   # a single tile
+    ("llm", {}, True, "max", "sample"),
+    ("llm", {}, True, "search", "sample"),
+]
+
+
+def run_attention(q, k, v, causal, mode):
+    qg, kg, vg = (gpu_quant(x, r, mode=mode) for x, r in ((q, "q"), (k, "k"), (v, "v")))
+    out, lse = sa.sa_attn_fwd(qg, kg, vg, causal, want_lse=True)
+    status_ok()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,shape,causal,mode,rows", ATTN_CASES)
+def test_attention_matches_oracle(name, shape, causal, mode, rows):
+    q, k, v = inputs(name, **shape)
+    B, H, N, D = q.shape
+    og, lg = run_attention(q, k, v, causal, mode)
+    ss = mode == "search"
+    qo, ko, vo = orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss), orc.quantize(v, "v", search=ss)
+    rr = sample_rows(N) if rows == "sample" else None
+    ref, lse_ref = orc.attention(qo, ko, vo, causal, rows=rr, want_lse=True)
+    got = og if rr is None else og[:, :, rr]
+    lse_got = lg if rr is None else lg[:, :, rr]
+    check_close(got, ref, f"attn {name}{shape} causal={causal} {mode}")
+    assert np.max(np.abs(lse_got - lse_ref)) < 1e-3
+    # quality against exact FP64 attention on the raw inputs (reported)
+    rq = rr if rr is not None else np.arange(N)
+    ex = exact_rows(q, k, v, causal, rq[:64], 1 / math.sqrt(D))
+    print("  quality vs exact (gpu): cos %.6f relL1 %.4f" % quality(got[:, :, :64], ex))
+    print("  quality vs exact (oracle): cos %.6f relL1 %.4f" % quality(ref[:, :, :64], ex))
+
+
+# ------------------------------------------------------------------ decode
+def run_decode(q, k, v):
+    B, Hkv, L, D = k.shape
+    kg = gpu_quant(k, "k")
+    vg = gpu_quant(v, "v")
+    out = sa.sa_attn_decode_kvfp4(q.cuda(), kg, vg)
+    status_ok()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [dict(B=2, Hq=8, Hkv=2, L=8192, D=128), dict(B=1, Hq=4, Hkv=4, L=4096 + 384, D=64),
+                                   dict(B=3, Hq=8, Hkv=1, L=256, D=128)])
+def test_decode_matches_oracle(shape):
+    q, k, v = wl.decode_inputs(**shape)
+    og = run_decode(q, k, v)
+    ko, vo = orc.quantize(k, "k"), orc.quantize(v, "v")
+    ref = orc.decode(q, ko, vo).reshape(og.shape)
+    check_close(og, ref, f"decode {shape}")
+
+
+def test_decode_full_size_sampled():
+    """Full decode workload (B32 Hq32 Hkv8 L32768 D128); all outputs from the
+    GPU, sampled (b, head) pairs from the oracle."""
+    q, k, v = wl.decode_inputs("decode")
+    og = run_decode(q, k, v)
+    ko, vo = orc.quantize(k, "k"), orc.quantize(v, "v")
+    pairs = np.array([0, 1, 5, 31, 32 * 7 + 3, 32 * 16 + 17, 32 * 31 + 30, 32 * 32 - 1], np.int32)
+    ref = orc.decode(q, ko, vo, pairs=pairs)
+    check_close(og.reshape(-1, 128)[pairs], ref, "decode full")
