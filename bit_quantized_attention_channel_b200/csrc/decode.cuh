@@ -29,14 +29,14 @@ constexpr int kDecN = 8;  // MMA N (query heads of a group, zero-padded)
 
 template <int D>
 struct DecSmem {
-    uint8_t k[128 * D / 2];    // K tile (A), D/2-byte swizzle
-    uint8_t v[128 * 64];       // V^T tile (A): 128 rows (channels >= D zero-filled), 64-byte swizzle
-    uint8_t ones[128 * 64];    // constant A operand: E2M1 1.0
-    uint8_t q[kDecN * D / 2];  // q^T (B): 8 rows, D/2-byte swizzle
-    uint8_t p[kDecN * 64];     // P^T (B): 8 rows x 128 keys, 64-byte swizzle
+    alignas(1024) uint8_t k[128 * D / 2];    // K tile (A), D/2-byte swizzle
+    alignas(1024) uint8_t v[128 * 64];       // V^T tile (A): 128 rows (channels >= D zero-filled), 64-byte swizzle
+    alignas(1024) uint8_t ones[128 * 64];    // constant A operand: E2M1 1.0
+    alignas(1024) uint8_t q[kDecN * D / 2];  // q^T (B): 8 rows, D/2-byte swizzle
+    alignas(1024) uint8_t p[kDecN * 64];     // P^T (B): 8 rows x 128 keys, 64-byte swizzle
     uint8_t ksf[D / 64 * 512];
     uint8_t vsf[2 * 512];
-    uint8_t qsf[D / 64 * 512];
+    alignas(16) uint8_t qsf[D / 64 * 512];
     uint8_t psf[2 * 512];
     uint8_t onesf[512];
     float red[4][kDecN];
@@ -250,8 +250,8 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     // ---- write this split's unnormalised O (lane = channel), l and m
     uint32_t o[kDecN], l[kDecN];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%9, %10, %11, %12, %13, %14, %15, %16}, [%17];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
         : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]),
           "=r"(l[0]), "=r"(l[1]), "=r"(l[2]), "=r"(l[3]), "=r"(l[4]), "=r"(l[5]), "=r"(l[6]), "=r"(l[7])

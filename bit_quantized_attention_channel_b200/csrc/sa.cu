@@ -45,6 +45,22 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
     return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor {d0 (contiguous, elements), d1, d2}; box {64, 128, 1} with
+// the 128-byte swizzle (one 128-byte row of 64 elements per box row).
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int rt_ck(int R, int C, int* RT, int* CK)
 {
     *RT = sa_cdiv(R, 128);
@@ -227,10 +243,6 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
                       const void* k_bf16_dev, const void* v_bf16_dev, const float* k_mean_dev, float* out_dev,
                       float* lse_dev, cudaStream_t stream)
 {
-    (void)q_bf16_dev;
-    (void)k_bf16_dev;
-    (void)v_bf16_dev;
-    (void)k_mean_dev;
     if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
     if (N % 32) return SA_ERR_INVALID_ARG;
@@ -241,15 +253,27 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     if (!aligned16(q_codes_dev) || !aligned16(k_codes_dev) || !aligned16(v_codes_dev) || !aligned16(q_scales_dev) ||
         !aligned16(k_scales_dev) || !aligned16(v_scales_dev) || !aligned16(out_dev))
         return SA_ERR_INVALID_ARG;
-    if (mask_dev) return SA_ERR_UNSUPPORTED;
+    const bool mixed = mask_dev != nullptr;
+    if (mixed && (!q_bf16_dev || !k_bf16_dev || !v_bf16_dev || !aligned16(q_bf16_dev) || !aligned16(k_bf16_dev) ||
+                  !aligned16(v_bf16_dev)))
+        return SA_ERR_INVALID_ARG;
     if (!(sm_scale > 0.0f)) sm_scale = 1.0f / sqrtf((float)D);
     const uint64_t BH = (uint64_t)B * H;
     const CUtensorMapSwizzle qsw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tqb, tkb, tvb;
     if (!make_map_u8(&tq, q_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
         !make_map_u8(&tk, k_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
         !make_map_u8(&tv, v_codes_dev, N / 2, D, BH, 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA_ERR_CUDA;
+    if (mixed) {
+        if (!make_map_bf16(&tqb, q_bf16_dev, D, N, BH) || !make_map_bf16(&tkb, k_bf16_dev, D, N, BH) ||
+            !make_map_bf16(&tvb, v_bf16_dev, D, N, BH))
+            return SA_ERR_CUDA;
+    } else {
+        tqb = tq;
+        tkb = tk;
+        tvb = tv;
+    }
     AttnParams p{};
     p.q_sf = q_scales_dev;
     p.k_sf = k_scales_dev;
@@ -265,21 +289,26 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     p.CKv = sa_cdiv(N, 64);
     p.causal = causal ? 1 : 0;
     p.sm_scale = sm_scale;
+    p.mask = mask_dev;
+    p.q_bf16 = (const uint16_t*)q_bf16_dev;
+    p.k_mean = k_mean_dev;
     dim3 grid(p.T, H, B);
-    // one CTA per SM (the CTA owns all 512 TMEM columns)
-    const int smem = 116 * 1024;
+#define SA_ATTN_LAUNCH(DD, MX)                                                                              \
+    do {                                                                                                    \
+        const int smem = MX ? (int)(((sizeof(AttnSmem<DD>) + 1023) & ~(size_t)1023) + sizeof(MixedSmem<DD>) + \
+                                    1024)                                                                   \
+                            : 116 * 1024; /* one CTA per SM: the CTA owns all 512 TMEM columns */          \
+        if (cudaFuncSetAttribute(attn_fwd_kernel<DD, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != \
+            cudaSuccess)                                                                                    \
+            return SA_ERR_CUDA;                                                                             \
+        attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
+    } while (0)
     if (D == 128) {
-        static_assert(sizeof(AttnSmem<128>) + 1024 <= 116 * 1024, "smem");
-        if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return SA_ERR_CUDA;
-        attn_fwd_kernel<128><<<grid, 128, smem, stream>>>(tq, tk, tv, p);
+        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_LAUNCH(128, false);
     } else {
-        if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return SA_ERR_CUDA;
-        attn_fwd_kernel<64><<<grid, 128, smem, stream>>>(tq, tk, tv, p);
+        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_LAUNCH(64, false);
     }
+#undef SA_ATTN_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
 }

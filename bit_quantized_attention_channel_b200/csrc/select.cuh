@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
                                                             int32_t* __restrict__ nsel)
 {
     __shared__ uint32_t hist[256];
-    __shared__ uint32_t s_prefix, s_need, s_digit;
+    __shared__ uint32_t s_prefix, s_need;
     __shared__ uint32_t scan[kTopkThreads];
     size_t bh = blockIdx.x;
     const float* sc = scores + bh * (size_t)T * T;
@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
                     if (acc + hist[d] >= need) break;
                     acc += hist[d];
                 }
-                s_digit = (uint32_t)d;
                 s_need = need - acc;
                 s_prefix = prefix | ((uint32_t)d << shift);
             }

@@ -207,3 +207,28 @@ SA_DEV void reg_fence(float (&v)[N])
     for (int i = 0; i < N; i++) asm volatile("" : "+f"(v[i])::"memory");
 }
 }  // namespace sa
+
+namespace sa {
+// Instruction descriptor of kind::f16 with bf16 A/B, FP32 accumulate.
+// b_mn_major: B stored MN-major (N contiguous), A always K-major here.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major)
+{
+    return (1u << 4)                          // D format: F32
+           | (1u << 7)                        // A format: BF16
+           | (1u << 10)                       // B format: BF16
+           | ((uint32_t)b_mn_major << 16)     // B major
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// D(tmem) (+)= A(smem) x B(smem) for 16-bit inputs (K = 16 per instruction).
+SA_DEV void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+}  // namespace sa
