@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "attn_ws.cuh"
 #include "decode.cuh"
 #include "quant.cuh"
 #include "select.cuh"
@@ -303,12 +304,21 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
             return SA_ERR_CUDA;                                                                             \
         attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
     } while (0)
+#define SA_ATTN_WS_LAUNCH(DD)                                                                               \
+    do {                                                                                                    \
+        const int smem = (int)sizeof(WsSmem<DD>) + 1024;                                                    \
+        if (cudaFuncSetAttribute(attn_fwd_ws_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != \
+            cudaSuccess)                                                                                    \
+            return SA_ERR_CUDA;                                                                             \
+        attn_fwd_ws_kernel<DD><<<grid, kWsThreads, smem, stream>>>(tq, tk, tv, p);                          \
+    } while (0)
     if (D == 128) {
-        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_LAUNCH(128, false);
+        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_WS_LAUNCH(128);
     } else {
-        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_LAUNCH(64, false);
+        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_WS_LAUNCH(64);
     }
 #undef SA_ATTN_LAUNCH
+#undef SA_ATTN_WS_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
 }

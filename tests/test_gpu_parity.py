@@ -262,3 +262,58 @@ def test_decode_full_size_sampled():
     pairs = np.array([0, 1, 5, 31, 32 * 7 + 3, 32 * 16 + 17, 32 * 31 + 30, 32 * 32 - 1], np.int32)
     ref = orc.decode(q, ko, vo, pairs=pairs)
     check_close(og.reshape(-1, 128)[pairs], ref, "decode full")
+
+
+# ------------------------------------------------------------------ mixed precision
+def run_mixed(q, k, v, causal, mask_cpu):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    qg, kg, vg = gpu_quant(q, "q"), gpu_quant(k, "k"), gpu_quant(v, "v")
+    out, lse = sa.sa_attn_fwd(qg, kg, vg, causal, mask=torch.from_numpy(mask_cpu).cuda(), q_bf16=qd, k_bf16=kd,
+                              v_bf16=vd, want_lse=True)
+    status_ok()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("mask_kind,causal,N,D", [("select", True, 1024, 128), ("select", False, 1024 + 256, 64),
+                                                  ("all", True, 512, 128), ("random", True, 640, 128),
+                                                  ("random", False, 416, 64)])
+def test_mixed_attention_matches_oracle(mask_kind, causal, N, D):
+    q, k, v = inputs("longctx", H=2, N=N, D=D)
+    T = (N + 127) // 128
+    if mask_kind == "select":
+        mask, _ = orc.thrift_select(q, k, causal, 1500)
+    elif mask_kind == "all":
+        mask = np.ones((1, 2, T, T), np.uint8)
+    else:
+        mask = (np.random.default_rng(3).random((1, 2, T, T)) < 0.3).astype(np.uint8)
+    og, lg = run_mixed(q, k, v, causal, mask)
+    qo, ko, vo = orc.quantize(q, "q"), orc.quantize(k, "k"), orc.quantize(v, "v")
+    ref, lse_ref = orc.attention(qo, ko, vo, causal, mask=mask, q_bf16=q, k_bf16=k, v_bf16=v, want_lse=True)
+    check_close(og, ref, f"mixed {mask_kind} causal={causal} N={N} D={D}")
+    assert np.max(np.abs(lg - lse_ref)) < 1e-3
+    # with no block selected the mixed kernel computes the NVFP4 result
+    if mask_kind == "select":
+        og0, _ = run_mixed(q, k, v, causal, np.zeros_like(mask))
+        of, _ = run_attention(q, k, v, causal, "max")
+        check_close(og0, of, "mixed kernel, empty mask vs NVFP4 kernel")
+
+
+def test_mixed_full_size_sampled():
+    """Long-context mixed workload (B1 H32 N65536 causal, 5 % bf16 blocks
+    chosen by the GPU selector, checked bit-exact against the oracle's)."""
+    q, k, v = inputs("longctx")
+    mg, _ = sa.sa_thrift_select(q.cuda(), k.cuda(), True, 500)
+    mask = mg.cpu().numpy()
+    mo, _ = orc.thrift_select(q, k, True, 500)
+    assert np.array_equal(mask, mo)
+    og, _ = run_mixed(q, k, v, True, mask)
+    qo, ko, vo = orc.quantize(q, "q"), orc.quantize(k, "k"), orc.quantize(v, "v")
+    rows = sample_rows(q.shape[2])
+    ref = orc.attention(qo, ko, vo, True, rows=rows, mask=mo, q_bf16=q, k_bf16=k, v_bf16=v)
+    check_close(og[:, :, rows], ref, "mixed full size")
+    # report the ThriftAttention-style gap recovery on these rows
+    fp4 = orc.attention(qo, ko, vo, True, rows=rows)
+    ex = exact_rows(q, k, v, True, rows, 1 / math.sqrt(q.shape[3]))
+    e4 = np.linalg.norm(fp4 - ex)
+    emx = np.linalg.norm(ref - ex)
+    print(f"  FP4->exact gap recovered by 5% bf16 blocks: {100 * (1 - emx / e4):.1f}%")
