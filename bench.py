@@ -99,30 +99,84 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def make_step(w, mode, q, k, v, stream):
-    """Returns step() running the whole path on device-resident inputs, and
-    the buffers it writes into (allocated once)."""
-    st = {}
+class Path:
+    """The hot path of one workload as two device-side phases (pre-pass,
+    attention), each captured once in a CUDA graph and replayed per step.
+    Inputs stay resident; outputs are written into the same buffers."""
 
-    def step(attn_events=None):
-        qq = sa.sa_quant_nvfp4(q, "q", mode=mode, out=st.get("q"), stream=stream)
-        kq = sa.sa_quant_nvfp4(k, "k", mode=mode, out=st.get("k"), stream=stream)
-        vq = sa.sa_quant_nvfp4(v, "v", mode=mode, out=st.get("v"), stream=stream)
-        st["q"], st["k"], st["v"] = qq, kq, vq
+    def __init__(self, w, mode, q, k, v):
+        self.w, self.mode, self.q, self.k, self.v = w, mode, q, k, v
+        self.st = {}
+
+    def prepass(self):
+        w, st = self.w, self.st
+        if w.kind == "decode":
+            return  # the KV cache is quantised once, before timing (it is a cache)
+        st["q"] = sa.sa_quant_nvfp4(self.q, "q", mode=self.mode, out=st.get("q"))
+        st["k"] = sa.sa_quant_nvfp4(self.k, "k", mode=self.mode, out=st.get("k"))
+        st["v"] = sa.sa_quant_nvfp4(self.v, "v", mode=self.mode, out=st.get("v"))
+        if w.thrift_bp:
+            st["mask"], _ = sa.sa_thrift_select(self.q, self.k, w.causal, w.thrift_bp)
+
+    def attention(self):
+        w, st = self.w, self.st
+        if w.kind == "decode":
+            st["o"] = sa.sa_attn_decode_kvfp4(self.q, st["kc"], st["vc"], out=st.get("o"))
+        elif w.thrift_bp:
+            st["o"] = sa.sa_attn_fwd(st["q"], st["k"], st["v"], w.causal, mask=st["mask"], q_bf16=self.q,
+                                     k_bf16=self.k, v_bf16=self.v, out=st.get("o"))
+        else:
+            st["o"] = sa.sa_attn_fwd(st["q"], st["k"], st["v"], w.causal, out=st.get("o"))
+        return st["o"]
+
+    def setup(self):
+        if self.w.kind == "decode":
+            self.st["kc"] = sa.sa_quant_nvfp4(self.k, "k")
+            self.st["vc"] = sa.sa_quant_nvfp4(self.v, "v")
+
+    def capture(self):
+        """Warm up eagerly, then capture both phases as CUDA graphs."""
+        self.setup()
+        for _ in range(2):
+            self.prepass()
+            self.attention()
+        torch.cuda.synchronize()
+        self.g_pre, self.g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_pre):
+            self.prepass()
+        with torch.cuda.graph(self.g_attn):
+            self.attention()
+        torch.cuda.synchronize()
+
+    def step(self, attn_events=None):
+        self.g_pre.replay()
         if attn_events:
-            attn_events[0].record(stream)
-        out = sa.sa_attn_fwd(qq, kq, vq, w.causal, out=st.get("o"), stream=stream)
+            attn_events[0].record()
+        self.g_attn.replay()
         if attn_events:
-            attn_events[1].record(stream)
-        st["o"] = out
-        return out
-
-    return step
+            attn_events[1].record()
+        return self.st["o"]
 
 
-def kernels_per_step(mode):
-    # q: amax + quant; k: stats + final + quant; v: amax + quant; attention: 1
-    return 2 + 3 + 2 + 1
+def kernels_per_step(w):
+    if w.kind == "decode":
+        return 3  # q amax, split kernel, combine
+    n = 2 + 3 + 2 + 1  # q: amax+quant, k: stats+final+quant, v: amax+quant, attention
+    if w.thrift_bp:
+        n += 3  # pool, score, top-k
+    return n
+
+
+def flops_of(w):
+    if w.kind == "decode":
+        return 4.0 * w.B * w.H * w.N * w.D
+    return w.flops()
+
+
+def hbm_bytes_decode(w):
+    """Algorithmic bytes of one decode: K and V codes + scales, q, out."""
+    kv = 2 * (w.B * w.Hkv * w.N * w.D // 2 + w.B * w.Hkv * w.N * w.D // 16)
+    return kv + w.B * w.H * w.D * (2 + 4)
 
 
 def cpu_baseline(w, mode, budget_s=20.0):
@@ -178,8 +232,14 @@ def run_reference(args, w, rank, world):
 
 
 def config_of(w, mode):
-    return {"workload": w.description, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "causal": w.causal,
-            "scale_mode": mode, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas"}
+    c = {"workload": w.description, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "causal": w.causal,
+         "scale_mode": mode, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
+         "launch": "CUDA graphs (pre-pass graph + attention graph per step)"}
+    if w.kind == "decode":
+        c["Hkv"] = w.Hkv
+    if w.thrift_bp:
+        c["bf16_block_budget_bp"] = w.thrift_bp
+    return c
 
 
 def main():
@@ -214,15 +274,20 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
 
-    q, k, v = (t.to(dev) for t in wl.prefill_inputs(w))
-    stream = torch.cuda.current_stream(dev)
-    step = make_step(w, args.mode, q, k, v, stream)
+    if w.kind == "decode":
+        q, k, v = (t.to(dev) for t in wl.decode_inputs(w))
+    else:
+        q, k, v = (t.to(dev) for t in wl.prefill_inputs(w))
+    path = Path(w, args.mode, q, k, v)
+    path.capture()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     for _ in range(args.warmup):
-        step()
+        flush.fill_(1)
+        path.step()
     torch.cuda.synchronize()
-    assert sa.sa_device_status() == 0
+    st = sa.sa_device_status()
+    assert st == 0, sa.STATUS[st]
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     aevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -233,9 +298,9 @@ def main():
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # evict L2 between steps (outside the step events)
-            evs[i][0].record(stream)
-            step(aevs[i])
-            evs[i][1].record(stream)
+            evs[i][0].record()
+            path.step(aevs[i])
+            evs[i][1].record()
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if pg:
@@ -249,22 +314,24 @@ def main():
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         ms, ms_attn = t.tolist()
 
-    # end to end through the C ABI from pinned host buffers
+    # end to end through the C ABI from pinned host buffers: copy the step's
+    # inputs in, run the path, copy the output back
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    hout = torch.empty(w.B, w.H, w.N, w.D, dtype=torch.float32).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    step_e2e = make_step(w, args.mode, dq, dk, dv, stream)
+    e2e_path = Path(w, args.mode, torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    e2e_path.st.update({kk: path.st[kk] for kk in ("kc", "vc") if kk in path.st})
+    hout = torch.empty(path.st["o"].shape, dtype=torch.float32).pin_memory()
+    h2d = [(e2e_path.q, hq)] if w.kind == "decode" else [(e2e_path.q, hq), (e2e_path.k, hk), (e2e_path.v, hv)]
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.fill_(i & 0xFF)
-        a.record(stream)
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        out = step_e2e()
+        a.record()
+        for dst, src in h2d:
+            dst.copy_(src, non_blocking=True)
+        e2e_path.prepass()
+        out = e2e_path.attention()
         hout.copy_(out, non_blocking=True)
-        b.record(stream)
+        b.record()
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
@@ -273,28 +340,37 @@ def main():
         t = torch.tensor([e2e], device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
         e2e = t.item()
+    h2d_bytes = sum(src.numel() * src.element_size() for _, src in h2d)
 
     if rank == 0:
         hbm, bf16, src = peaks()
         fp4_peak = bf16 * 4.0  # dense FP4 = 4x dense bf16 (nominal ratio 9 / 2.25)
-        flops = w.flops()
-        achieved = flops / (ms_attn * 1e-3) / 1e12
+        flops = flops_of(w)
+        if w.kind == "decode":
+            gbs = hbm_bytes_decode(w) / (ms_attn * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "decode_kernel<128> + combine", "achieved": gbs, "peak": hbm,
+                    "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{src} copy bandwidth",
+                    "traffic": None, "ms_per_launch": ms_attn, "algorithmic_bytes": hbm_bytes_decode(w)}
+        else:
+            achieved = flops / (ms_attn * 1e-3) / 1e12
+            kname = "attn_fwd_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_ws_kernel<128>"
+            roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                    "frac": achieved / fp4_peak,
+                    "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
+                    "traffic": None, "ms_per_launch": ms_attn}
         line = {
             "metric": METRIC, "value": world * flops / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
             "config": config_of(w, args.mode),
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
-                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
-                         "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
-                         "traffic": None, "ms_per_launch": ms_attn},
+            "roofline": roof,
             "e2e": {"value": world * flops / (e2e * 1e-3) / 1e12, "unit": "TOPS",
-                    "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": hout.numel() * 4},
-            "gpu_launches": kernels_per_step(args.mode) * args.steps,
+                    "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": hout.numel() * 4},
+            "gpu_launches": kernels_per_step(w) * args.steps,
             "clocks": clk.summary(),
             "wall_s": t_wall,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and w.kind != "decode":
             line["cpu_baseline"] = cpu_baseline(w, args.mode)
         print(json.dumps(line), flush=True)
     if pg:

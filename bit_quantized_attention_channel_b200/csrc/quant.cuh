@@ -15,7 +15,7 @@
 //   kfinal_kernel      per (b,h,channel): tile partials in tile order -> mean;
 //                      amax of K - mean from max/min (rounding is monotone).
 //   quant_rows_kernel  Q/K: one thread per 16-channel block.
-//   quant_v_kernel     V: one thread per 16-token block of one channel.
+//   quant_v_kernel     V: one thread per 16-token block of four channels.
 #pragma once
 
 #include "common.cuh"
@@ -99,12 +99,26 @@ SA_DEV void quant16(const float (&xt)[16], int f_lo, int f_hi, uint32_t& w0, uin
 // ---------------------------------------------------------------------------
 
 // max |x| over n16 groups of 8 bf16; raises SA_ERR_NONFINITE on inf/NaN.
+// Four independent 16-byte loads per thread and iteration.
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict__ x, size_t n16,
                                                         unsigned* __restrict__ amax_word)
 {
     uint32_t m = 0;
-    size_t stride = (size_t)gridDim.x * blockDim.x;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += stride) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) v[u] = __ldcs(x + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
+        }
+    }
+    for (; i < n16; i += stride) {
         uint4 v = __ldcs(x + i);
         m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
         m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
@@ -144,17 +158,23 @@ __global__ void __launch_bounds__(256) kstats_kernel(const uint32_t* __restrict_
     double s0 = 0.0, s1 = 0.0;
     float mx0 = -INFINITY, mx1 = -INFINITY, mn0 = INFINITY, mn1 = INFINITY;
     bool bad = false;
-#pragma unroll 8
-    for (int r = 0; r < rows; r++) {
-        uint32_t w = __ldcs(p + (size_t)r * P);
-        float a = bf16_bits_to_f32(w & 0xFFFFu), b = bf16_bits_to_f32(w >> 16);
-        bad |= !isfinite(a) || !isfinite(b);
-        s0 = __dadd_rn(s0, (double)a);
-        s1 = __dadd_rn(s1, (double)b);
-        mx0 = fmaxf(mx0, a);
-        mx1 = fmaxf(mx1, b);
-        mn0 = fminf(mn0, a);
-        mn1 = fminf(mn1, b);
+    for (int r0b = 0; r0b < rows; r0b += 16) {
+        uint32_t w[16];
+#pragma unroll
+        for (int u = 0; u < 16; u++) w[u] = r0b + u < rows ? __ldcs(p + (size_t)(r0b + u) * P) : 0u;
+        const int nr = min(16, rows - r0b);
+#pragma unroll
+        for (int u = 0; u < 16; u++) {
+            if (u >= nr) break;
+            float a = bf16_bits_to_f32(w[u] & 0xFFFFu), b = bf16_bits_to_f32(w[u] >> 16);
+            bad |= !isfinite(a) || !isfinite(b);
+            s0 = __dadd_rn(s0, (double)a);  // tokens in ascending order
+            s1 = __dadd_rn(s1, (double)b);
+            mx0 = fmaxf(mx0, a);
+            mx1 = fmaxf(mx1, b);
+            mn0 = fminf(mn0, a);
+            mn1 = fminf(mn1, b);
+        }
     }
     if (bad) sa_raise(SA_ERR_NONFINITE);
     size_t o = (bh * T + tile) * D + 2 * cp;
@@ -179,11 +199,23 @@ __global__ void __launch_bounds__(128) kfinal_kernel(const double* __restrict__ 
     if (c < D) {
         double total = 0.0;
         float mx = -INFINITY, mn = INFINITY;
-        for (int t = 0; t < T; t++) {
-            size_t o = (bh * T + t) * D + c;
-            total = __dadd_rn(total, psum[o]);
-            mx = fmaxf(mx, pmax[o]);
-            mn = fminf(mn, pmin[o]);
+        for (int t0 = 0; t0 < T; t0 += 8) {
+            double ps[8];
+            float px[8], pn[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const size_t o = (bh * T + min(t0 + u, T - 1)) * D + c;
+                ps[u] = psum[o];
+                px[u] = pmax[o];
+                pn[u] = pmin[o];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                if (t0 + u >= T) break;
+                total = __dadd_rn(total, ps[u]);  // tiles in ascending order
+                mx = fmaxf(mx, px[u]);
+                mn = fminf(mn, pn[u]);
+            }
         }
         float mu = __double2float_rn(__ddiv_rn(total, (double)N));
         kmean[bh * D + c] = mu;
@@ -241,41 +273,52 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     }
 }
 
-// V: thread per (channel, 16-token block); codes land in [B,H,D,N/2].
-// nblk = B*H*(N/16)*D, channel fastest so a warp reads whole row segments.
+// V: thread per (4 channels, 16-token block); codes land in [B,H,D,N/2].
+// nblk4 = B*H*(N/16)*(D/4), channel group fastest so a warp reads 256
+// contiguous bytes of each token row.
 template <bool SEARCH>
-__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ x, size_t nblk, int N, int D,
+__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ x, size_t nblk4, int N, int D,
                                                       const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                       int8_t* __restrict__ ss_off, float* __restrict__ g_out)
 {
     float g, inv_g;
     tensor_scale(__uint_as_float(*amax_word), g, inv_g);
-    size_t stride = (size_t)gridDim.x * blockDim.x;
-    size_t b0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t b0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (b0 == 0) {
         g_out[0] = g;
         g_out[1] = inv_g;
     }
-    const int NBT = N / 16;
+    const int NBT = N / 16, D4 = D / 4;
     const int RT = (D + 127) / 128, CK = (N + 63) / 64;
-    for (size_t b = b0; b < nblk; b += stride) {
-        int c = (int)(b % D);
-        size_t rest = b / D;
-        int nb = (int)(rest % NBT);
-        size_t bh = rest / NBT;
-        const uint16_t* p = x + (bh * N + (size_t)nb * 16) * D + c;
-        float xt[16];
+    for (size_t b = b0; b < nblk4; b += stride) {
+        const int c0 = (int)(b % D4) * 4;
+        const size_t rest = b / D4;
+        const int nb = (int)(rest % NBT);
+        const size_t bh = rest / NBT;
+        const uint16_t* p = x + (bh * N + (size_t)nb * 16) * D + c0;
+        uint2 w[16];
 #pragma unroll
-        for (int i = 0; i < 16; i++) xt[i] = __fmul_rn(bf16_bits_to_f32(__ldcs(p + (size_t)i * D)), inv_g);
-        uint32_t c0, c1, sc;
-        int off;
-        quant16<SEARCH>(xt, f_lo, f_hi, c0, c1, sc, off);
-        size_t crow = bh * D + c;
-        *reinterpret_cast<uint2*>(codes + crow * (N / 2) + (size_t)nb * 8) = make_uint2(c0, c1);
-        size_t atom = (bh * RT + (size_t)(c >> 7)) * CK + (size_t)(nb >> 2);
-        scales[atom * 512 + sf_atom_offset((uint32_t)(c & 127), (uint32_t)(nb & 3))] = (uint8_t)sc;
-        if (ss_off) ss_off[crow * NBT + nb] = (int8_t)off;
+        for (int i = 0; i < 16; i++) w[i] = __ldcs(reinterpret_cast<const uint2*>(p + (size_t)i * D));
+#pragma unroll
+        for (int cc = 0; cc < 4; cc++) {
+            float xt[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const uint32_t word = cc < 2 ? w[i].x : w[i].y;
+                xt[i] = __fmul_rn(bf16_bits_to_f32((word >> (16 * (cc & 1))) & 0xFFFFu), inv_g);
+            }
+            uint32_t q0, q1, sc;
+            int off;
+            quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off);
+            const int c = c0 + cc;
+            const size_t crow = bh * D + c;
+            *reinterpret_cast<uint2*>(codes + crow * (N / 2) + (size_t)nb * 8) = make_uint2(q0, q1);
+            const size_t atom = (bh * RT + (size_t)(c >> 7)) * CK + (size_t)(nb >> 2);
+            scales[atom * 512 + sf_atom_offset((uint32_t)(c & 127), (uint32_t)(nb & 3))] = (uint8_t)sc;
+            if (ss_off) ss_off[crow * NBT + nb] = (int8_t)off;
+        }
     }
 }
 

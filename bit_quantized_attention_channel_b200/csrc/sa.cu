@@ -171,13 +171,13 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
 
     const bool ss = mode == SA_SCALE_SEARCH;
     if (role == SA_ROLE_V) {
-        size_t nblk = BH * (N / 16) * D;
-        int grid = grid_for(nblk, 256);
+        size_t nblk4 = BH * (N / 16) * (D / 4);
+        int grid = grid_for(nblk4, 256);
         if (ss)
-            quant_v_kernel<true><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk, N, D, w.amax, f_lo, f_hi,
+            quant_v_kernel<true><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk4, N, D, w.amax, f_lo, f_hi,
                                                            codes_dev, scales_dev, ss_off_dev, g_dev);
         else
-            quant_v_kernel<false><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk, N, D, w.amax, f_lo, f_hi,
+            quant_v_kernel<false><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk4, N, D, w.amax, f_lo, f_hi,
                                                             codes_dev, scales_dev, ss_off_dev, g_dev);
     } else {
         size_t nblk = BH * N * (D / 16);
@@ -299,17 +299,25 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
         const int smem = MX ? (int)(((sizeof(AttnSmem<DD>) + 1023) & ~(size_t)1023) + sizeof(MixedSmem<DD>) + \
                                     1024)                                                                   \
                             : 116 * 1024; /* one CTA per SM: the CTA owns all 512 TMEM columns */          \
-        if (cudaFuncSetAttribute(attn_fwd_kernel<DD, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != \
-            cudaSuccess)                                                                                    \
-            return SA_ERR_CUDA;                                                                             \
+        static int attr_done = 0; /* attribute set once, outside any stream capture */                    \
+        if (!attr_done) {                                                                                   \
+            if (cudaFuncSetAttribute(attn_fwd_kernel<DD, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                     smem) != cudaSuccess)                                                  \
+                return SA_ERR_CUDA;                                                                         \
+            attr_done = 1;                                                                                  \
+        }                                                                                                   \
         attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
     } while (0)
 #define SA_ATTN_WS_LAUNCH(DD)                                                                               \
     do {                                                                                                    \
         const int smem = (int)sizeof(WsSmem<DD>) + 1024;                                                    \
-        if (cudaFuncSetAttribute(attn_fwd_ws_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != \
-            cudaSuccess)                                                                                    \
-            return SA_ERR_CUDA;                                                                             \
+        static int attr_done = 0;                                                                           \
+        if (!attr_done) {                                                                                   \
+            if (cudaFuncSetAttribute(attn_fwd_ws_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                     smem) != cudaSuccess)                                                  \
+                return SA_ERR_CUDA;                                                                         \
+            attr_done = 1;                                                                                  \
+        }                                                                                                   \
         attn_fwd_ws_kernel<DD><<<grid, kWsThreads, smem, stream>>>(tq, tk, tv, p);                          \
     } while (0)
     if (D == 128) {
@@ -380,15 +388,23 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
     dim3 grid(nsplit, Hkv, B);
     if (D == 128) {
         const int smem = (int)sizeof(DecSmem<128>) + 1024;
-        if (cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return SA_ERR_CUDA;
+        static int attr_done = 0;
+        if (!attr_done) {
+            if (cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return SA_ERR_CUDA;
+            attr_done = 1;
+        }
         decode_kernel<128><<<grid, 128, smem, stream>>>(tk, tv, p);
     } else {
         const int smem = (int)sizeof(DecSmem<64>) + 1024;
-        if (cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return SA_ERR_CUDA;
+        static int attr_done = 0;
+        if (!attr_done) {
+            if (cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+                return SA_ERR_CUDA;
+            attr_done = 1;
+        }
         decode_kernel<64><<<grid, 128, smem, stream>>>(tk, tv, p);
     }
     SA_CHECK_LAUNCH();
