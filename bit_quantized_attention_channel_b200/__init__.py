@@ -53,6 +53,8 @@ def lib():
         L.sa_quant_workspace_size.argtypes, L.sa_quant_workspace_size.restype = [I, I, I, I, I], Z
         L.sa_quant_nvfp4.argtypes = [P, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, Z, P]
         L.sa_quant_nvfp4.restype = I
+        L.sa_quant_nvfp4_noalloc.argtypes = [P, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P]
+        L.sa_quant_nvfp4_noalloc.restype = I
         L.sa_select_workspace_size.argtypes, L.sa_select_workspace_size.restype = [I, I, I, I], Z
         L.sa_thrift_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P, Z, P]
         L.sa_thrift_select.restype = I

@@ -414,3 +414,53 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// sa_quant_nvfp4_noalloc: the pre-pass with library-owned scratch.
+// The scratch is a file-scope device array in this module (every GPU that
+// loads the module keeps it until the process exits).  Host code cannot pass
+// the array's name to a kernel (on the host it names a stand-in object, not
+// device memory), so each device's address is looked up once with
+// cudaGetSymbolAddress while that device is current.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+extern "C" sa_status sa_quant_nvfp4_noalloc(const void* x_dev, int B, int H, int N, int D, sa_role role, int smooth,
+                                            sa_scale_mode mode, int f_lo, int f_hi, uint8_t* codes_dev,
+                                            uint8_t* scales_dev, float* g_dev, float* k_mean_dev,
+                                            int8_t* ss_off_dev, cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return SA_ERR_INVALID_ARG;
+    if (role != SA_ROLE_Q && role != SA_ROLE_K && role != SA_ROLE_V) return SA_ERR_INVALID_ARG;
+    // size check first: nothing is launched or dereferenced for a call that
+    // does not fit the scratch
+    if (sa_quant_workspace_size(B, H, N, D, role) > kNoAllocScratchBytes) return SA_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return SA_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+                cudaGetLastError();
+                return SA_ERR_CUDA;
+            }
+            g_noalloc_ptr[dev] = ptr;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // the allocating entry point clears the parts of the workspace that must
+    // start at zero (the amax word) on `stream` before its kernels use them
+    return sa_quant_nvfp4(x_dev, B, H, N, D, role, smooth, mode, f_lo, f_hi, codes_dev, scales_dev, g_dev,
+                          k_mean_dev, ss_off_dev, scratch, kNoAllocScratchBytes, stream);
+}

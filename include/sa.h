@@ -119,6 +119,32 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
                          cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * sa_quant_nvfp4_noalloc -- sa_quant_nvfp4 without a caller workspace.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory: hosts whose device memory is all owned
+ * by a fixed pool or an external allocator, plug-ins that are handed buffers
+ * but no allocator, and latency-critical loops where the device-wide
+ * synchronisation of cudaMalloc/cudaFree is not allowed.
+ * Such a caller passes only its inputs and outputs (same meaning, layout and
+ * results as sa_quant_nvfp4); the scratch is an 8 MiB array inside libsa,
+ * held on every GPU that loads the library until the process exits.
+ *  - Limit: sa_quant_workspace_size(B,H,N,D,role) must be <= 8 MiB, else
+ *    SA_ERR_WORKSPACE is returned before anything is launched.  Q and V need
+ *    256 bytes; K needs about 16*B*H*ceil(N/128)*D + 4*B*H*D bytes more
+ *    (e.g. B*H*ceil(N/128) <= 3900 at D = 128).
+ *  - The first call on a device looks up the scratch address for that
+ *    device (cudaGetSymbolAddress, with the device current); make that first
+ *    call before any stream capture.
+ *  - Calls share the scratch and it keeps the last call's contents; the call
+ *    clears what must start at zero.  Calls that overlap on the GPU (for
+ *    example on two streams at once) race: serialise them.
+ *  - Allocates nothing: no cudaMalloc/cudaFree and no allocating library.
+ * ------------------------------------------------------------------------ */
+sa_status sa_quant_nvfp4_noalloc(const void* x_dev, int B, int H, int N, int D, sa_role role, int smooth,
+                                 sa_scale_mode mode, int f_lo, int f_hi, uint8_t* codes_dev, uint8_t* scales_dev,
+                                 float* g_dev, float* k_mean_dev, int8_t* ss_off_dev, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * sa_thrift_select -- pick the high-precision (query tile, key tile) blocks.
  * "ThriftAttention: 5%의 연산량으로 90%의 품질 유지" (the share of blocks and
  * the joint softmax; the page does not define the selector, so a mean-pooled
