@@ -46,57 +46,86 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed
+    region: an NVML polling thread (about one sample per millisecond), else
+    nvidia-smi at its fastest rate."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, cuda_index):
+        self.cuda_index = cuda_index
+        self.samples = []  # (sm_mhz, reason bits)
+        self.max_mhz = None
+        self.stop = threading.Event()
+        self.ready = threading.Event()
+        self.thread = None
+        self.source = None
+
+    def _handle(self, nv):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _poll_nvml(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(get_reasons(h))))
+            except Exception:
+                pass
+            self.ready.set()
+            time.sleep(0.001)
+
+    def _poll_smi(self):
+        q = "clocks.sm,clocks.max.sm," + ",".join("clocks_event_reasons." + n for n, _ in self.REASONS)
+        proc = subprocess.Popen(["nvidia-smi", "-i", str(self.cuda_index), f"--query-gpu={q}",
+                                 "--format=csv,noheader,nounits", "-lms", "10"], stdout=subprocess.PIPE,
+                                stderr=subprocess.DEVNULL, text=True)
+        self.ready.set()
+        for line in proc.stdout:
+            p = [x.strip() for x in line.split(",")]
+            if self.stop.is_set():
+                break
+            try:
+                bits = sum(bit for (_, bit), v in zip(self.REASONS, p[2:]) if v.lower() == "active")
+                self.samples.append((float(p[0]), bits))
+                self.max_mhz = float(p[1])
+            except (ValueError, IndexError):
+                continue
+        proc.terminate()
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml"
         except Exception:
-            self.proc = None
+            self.thread = threading.Thread(target=self._poll_smi, daemon=True)
+            self.source = "nvidia-smi"
+        self.thread.start()
+        self.ready.wait(timeout=5)
+        self.samples.clear()  # keep only samples taken inside the region
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            p = [x.strip() for x in ln.split(",")]
-            if len(p) < 7:
-                continue
-            try:
-                sm.append(float(p[0]))
-                mx = max(mx, float(p[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, p[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [c for c, _ in self.samples]
+        bits = 0
+        for _, b in self.samples:
+            bits |= b
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": [n for n, bit in self.REASONS if bits & bit], "samples": len(sm), "source": self.source}
 
 
 class Path:
@@ -245,7 +274,7 @@ def config_of(w, mode):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llm")
     ap.add_argument("--mode", default="max", choices=["max", "search"])
@@ -353,7 +382,7 @@ def main():
                     "traffic": None, "ms_per_launch": ms_attn, "algorithmic_bytes": hbm_bytes_decode(w)}
         else:
             achieved = flops / (ms_attn * 1e-3) / 1e12
-            kname = "attn_fwd_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_ws_kernel<128>"
+            kname = "attn_fwd_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_pp_kernel<128>"
             roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                     "frac": achieved / fp4_peak,
                     "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 
+#include "attn_pp.cuh"
 #include "attn_ws.cuh"
 #include "decode.cuh"
 #include "quant.cuh"
@@ -320,13 +321,26 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
         }                                                                                                   \
         attn_fwd_ws_kernel<DD><<<grid, kWsThreads, smem, stream>>>(tq, tk, tv, p);                          \
     } while (0)
+#define SA_ATTN_PP_LAUNCH(DD)                                                                               \
+    do {                                                                                                    \
+        const int smem = (int)sizeof(PpSmem<DD>) + 1024;                                                    \
+        static int attr_done = 0;                                                                           \
+        if (!attr_done) {                                                                                   \
+            if (cudaFuncSetAttribute(attn_fwd_pp_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                     smem) != cudaSuccess)                                                  \
+                return SA_ERR_CUDA;                                                                         \
+            attr_done = 1;                                                                                  \
+        }                                                                                                   \
+        attn_fwd_pp_kernel<DD><<<dim3((p.T + 1) / 2, H, B), kPpThreads, smem, stream>>>(tq, tk, tv, p);      \
+    } while (0)
     if (D == 128) {
-        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_WS_LAUNCH(128);
+        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_PP_LAUNCH(128);
     } else {
-        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_WS_LAUNCH(64);
+        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_PP_LAUNCH(64);
     }
 #undef SA_ATTN_LAUNCH
 #undef SA_ATTN_WS_LAUNCH
+#undef SA_ATTN_PP_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
 }

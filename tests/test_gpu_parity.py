@@ -201,6 +201,7 @@ ATTN_CASES = [
     ("tiny", {"N": 416, "D": 128}, True, "max", None),  # ragged last tile (416 = 3*128 + 32)
     ("tiny", {"N": 352}, False, "search", None),       # ragged, D = 64
     ("tiny", {"N": 128, "H": 1}, True, "max", None),   # a single tile
+    ("tiny", {"N": 640, "D": 128}, True, "max", None),  # odd tile count: last CTA has one query tile
     ("llm", {}, True, "max", "sample"),
     ("llm", {}, True, "search", "sample"),
 ]
