@@ -187,6 +187,19 @@ def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.
 
 
 # --------------------------------------------------------------------- layouts
+def codes_to_logical(codes, B: int, H: int, N: int, D: int, role: str):
+    """Codes in the logical row-major layout: [B,H,N,D/2] for Q/K (already
+    so stored) and [B,H,D,N/2] for V, whose storage is 128-token tiles
+    [B,H,ceil(N/128),D,64] (include/sa.h).  Pure index permutation."""
+    if role != "v":
+        return codes.reshape(B, H, N, D // 2)
+    NT = (N + 127) // 128
+    a = codes.reshape(B, H, NT, D, 64).permute(0, 1, 3, 2, 4) if hasattr(codes, "permute") else \
+        codes.reshape(B, H, NT, D, 64).transpose(0, 1, 3, 2, 4)
+    a = a.reshape(B, H, D, NT * 64)[:, :, :, : N // 2]
+    return a.contiguous() if hasattr(a, "contiguous") else a
+
+
 def scales_to_logical(scales, B: int, H: int, N: int, D: int, role: str):
     """Unpack the tensor-core atom layout of scale bytes (include/sa.h) into
     the logical row-major [B,H,R,C/16] layout (R, C = N, D for Q/K and D, N for

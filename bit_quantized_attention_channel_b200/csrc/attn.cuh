@@ -262,7 +262,7 @@ SA_DEV bool attn_body(AttnSmem<D>& s, MixedSmem<D>* mx, const CUtensorMap* tm_q,
             mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
             tma_load_3d(s.k, tm_k, &s.tma_bar, 0, u * 128, bh);
             bulk_load(s.ksf, p.k_sf + ((size_t)bh * p.T + u) * KB * 512, KB * 512, &s.tma_bar);
-            tma_load_3d(s.v, tm_v, &s.tma_bar, u * 64, 0, bh);
+            tma_load_3d(s.v, tm_v, &s.tma_bar, 0, u * D, bh);
             bulk_load(s.vsf, p.v_sf + ((size_t)bh * p.CKv + 2 * u) * 512, kblocks * 512, &s.tma_bar);
         }
         if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;

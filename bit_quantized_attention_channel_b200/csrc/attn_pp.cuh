@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 mbar_expect_tx(&s.kv_full[st], 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
                 tma_load_3d(s.k[st], &tm_k, &s.kv_full[st], 0, u * 128, bh);
                 bulk_load(s.ksf[st], p.k_sf + ((size_t)bh * p.T + u) * KB * 512, KB * 512, &s.kv_full[st]);
-                tma_load_3d(s.v[st], &tm_v, &s.kv_full[st], u * 64, 0, bh);
+                tma_load_3d(s.v[st], &tm_v, &s.kv_full[st], 0, u * D, bh);
                 bulk_load(s.vsf[st], p.v_sf + ((size_t)bh * p.CKv + 2 * u) * 512, kblocks * 512, &s.kv_full[st]);
             }
         }

@@ -30,7 +30,7 @@ constexpr int kDecN = 8;  // MMA N (query heads of a group, zero-padded)
 template <int D>
 struct DecSmem {
     alignas(1024) uint8_t k[128 * D / 2];    // K tile (A), D/2-byte swizzle
-    alignas(1024) uint8_t v[128 * 64];       // V^T tile (A): 128 rows (channels >= D zero-filled), 64-byte swizzle
+    alignas(1024) uint8_t v[128 * 64];       // V^T tile (A): 128 rows (rows >= D stay zero), 64-byte swizzle
     alignas(1024) uint8_t ones[128 * 64];    // constant A operand: E2M1 1.0
     alignas(1024) uint8_t q[kDecN * D / 2];  // q^T (B): 8 rows, D/2-byte swizzle
     alignas(1024) uint8_t p[kDecN * 64];     // P^T (B): 8 rows x 128 keys, 64-byte swizzle
@@ -121,10 +121,10 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     for (int u = 0; u < ntiles; u++) {
         const int ktile = key0 / 128 + u;
         if (tid == 0) {
-            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + 128 * 64 + 2 * 512);
+            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + 2 * 512);
             tma_load_3d(s.k, tm_k, &s.tma_bar, 0, ktile * 128, bhk);
             bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + ktile) * KB * 512, KB * 512, &s.tma_bar);
-            tma_load_3d(s.v, tm_v, &s.tma_bar, ktile * 64, 0, bhk);
+            tma_load_3d(s.v, tm_v, &s.tma_bar, 0, ktile * D, bhk);
             bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * ktile) * 512, 2 * 512, &s.tma_bar);
         }
         if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
     for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
     for (int i = tid; i < kDecN * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.p)[i] = 0u;
     for (int i = tid; i < 2 * 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.psf)[i] = 0u;
+    for (int i = D * 64 / 4 + tid; i < 128 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.v)[i] = 0u;
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();

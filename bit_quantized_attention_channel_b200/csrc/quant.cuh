@@ -273,7 +273,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
     }
 }
 
-// V: thread per (4 channels, 16-token block); codes land in [B,H,D,N/2].
+// V: thread per (4 channels, 16-token block); codes land in 128-token tiles
+// [B,H,ceil(N/128),D,64] (each tile's V^T block is one contiguous D x 64-byte
+// region, the operand of one P V MMA).
 // nblk4 = B*H*(N/16)*(D/4), channel group fastest so a warp reads 256
 // contiguous bytes of each token row.
 template <bool SEARCH>
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict
         g_out[1] = inv_g;
     }
     const int NBT = N / 16, D4 = D / 4;
-    const int RT = (D + 127) / 128, CK = (N + 63) / 64;
+    const int RT = (D + 127) / 128, CK = (N + 63) / 64, NT = (N + 127) / 128;
     for (size_t b = b0; b < nblk4; b += stride) {
         const int c0 = (int)(b % D4) * 4;
         const size_t rest = b / D4;
@@ -314,7 +316,8 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict
             quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off);
             const int c = c0 + cc;
             const size_t crow = bh * D + c;
-            *reinterpret_cast<uint2*>(codes + crow * (N / 2) + (size_t)nb * 8) = make_uint2(q0, q1);
+            *reinterpret_cast<uint2*>(codes + ((bh * NT + (size_t)(nb >> 3)) * D + c) * 64 + (size_t)(nb & 7) * 8) =
+                make_uint2(q0, q1);
             const size_t atom = (bh * RT + (size_t)(c >> 7)) * CK + (size_t)(nb >> 2);
             scales[atom * 512 + sf_atom_offset((uint32_t)(c & 127), (uint32_t)(nb & 3))] = (uint8_t)sc;
             if (ss_off) ss_off[crow * NBT + nb] = (int8_t)off;

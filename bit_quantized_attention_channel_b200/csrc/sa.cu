@@ -7,7 +7,6 @@
 #include <cstring>
 
 #include "attn_pp.cuh"
-#include "attn_ws.cuh"
 #include "decode.cuh"
 #include "quant.cuh"
 #include "select.cuh"
@@ -106,8 +105,8 @@ sa_status sa_device_status(cudaStream_t stream, int reset)
 
 size_t sa_codes_bytes(int B, int H, int N, int D, sa_role role)
 {
-    (void)role;
     if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    if (role == SA_ROLE_V) return (size_t)B * H * sa_cdiv(N, 128) * D * 64;  // whole 128-token tiles
     return (size_t)B * H * N * D / 2;
 }
 
@@ -265,7 +264,7 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     CUtensorMap tq, tk, tv, tqb, tkb, tvb;
     if (!make_map_u8(&tq, q_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
         !make_map_u8(&tk, k_codes_dev, D / 2, N, BH, D / 2, 128, qsw) ||
-        !make_map_u8(&tv, v_codes_dev, N / 2, D, BH, 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map_u8(&tv, v_codes_dev, 64, (uint64_t)D * sa_cdiv(N, 128), BH, 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA_ERR_CUDA;
     if (mixed) {
         if (!make_map_bf16(&tqb, q_bf16_dev, D, N, BH) || !make_map_bf16(&tkb, k_bf16_dev, D, N, BH) ||
@@ -309,18 +308,6 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
         }                                                                                                   \
         attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
     } while (0)
-#define SA_ATTN_WS_LAUNCH(DD)                                                                               \
-    do {                                                                                                    \
-        const int smem = (int)sizeof(WsSmem<DD>) + 1024;                                                    \
-        static int attr_done = 0;                                                                           \
-        if (!attr_done) {                                                                                   \
-            if (cudaFuncSetAttribute(attn_fwd_ws_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                     smem) != cudaSuccess)                                                  \
-                return SA_ERR_CUDA;                                                                         \
-            attr_done = 1;                                                                                  \
-        }                                                                                                   \
-        attn_fwd_ws_kernel<DD><<<grid, kWsThreads, smem, stream>>>(tq, tk, tv, p);                          \
-    } while (0)
 #define SA_ATTN_PP_LAUNCH(DD)                                                                               \
     do {                                                                                                    \
         const int smem = (int)sizeof(PpSmem<DD>) + 1024;                                                    \
@@ -339,7 +326,6 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
         if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_PP_LAUNCH(64);
     }
 #undef SA_ATTN_LAUNCH
-#undef SA_ATTN_WS_LAUNCH
 #undef SA_ATTN_PP_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
@@ -381,7 +367,7 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
     const CUtensorMapSwizzle ksw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
     CUtensorMap tk, tv;
     if (!make_map_u8(&tk, k_codes_dev, D / 2, L, BHk, D / 2, 128, ksw) ||
-        !make_map_u8(&tv, v_codes_dev, L / 2, D, BHk, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map_u8(&tv, v_codes_dev, 64, (uint64_t)D * sa_cdiv(L, 128), BHk, 64, D, CU_TENSOR_MAP_SWIZZLE_64B))
         return SA_ERR_CUDA;
     DecParams p{};
     p.q = (const uint16_t*)q_dev;

@@ -34,9 +34,13 @@
  *    scale); an all-zero tensor has g = 1.
  *  - codes: E2M1 nibbles, two per byte, even element in the low nibble.
  *    Q and K: [B, H, N, D/2] (blocks of 16 consecutive channels of a token).
- *    V:       [B, H, D, N/2] (blocks of 16 consecutive tokens of a channel --
- *    the key axis is the reduction axis of P V, the only axis a block-scaled
- *    MMA can scale along).
+ *    V:       blocks of 16 consecutive tokens of a channel (the key axis is
+ *    the reduction axis of P V, the only axis a block-scaled MMA can scale
+ *    along), stored in 128-token tiles [B, H, ceil(N/128), D, 64]: byte
+ *    ((b*H + h)*ceil(N/128) + n/128)*D*64 + d*64 + (n%128)/2 holds tokens n, n+1
+ *    (n even) of channel d, so each tile's V^T block is one contiguous
+ *    D x 64-byte region.  Bytes past token N in the last tile are unspecified.
+ *    Size: sa_codes_bytes().
  *  - scales: E4M3 bytes, one per block, in the tensor-core "atom" layout.
  *    View each (b, h) slice as a matrix with R rows and C block-running
  *    columns (Q, K: R = N, C = D; V: R = D, C = N).  Rows are grouped into

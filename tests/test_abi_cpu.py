@@ -40,6 +40,9 @@ def test_status_strings(L):
 def test_buffer_sizes(L):
     # Q/K: codes B*H*N*D/2; scales: 512-byte atoms per (128 rows, 64 columns)
     assert L.sa_codes_bytes(2, 16, 4096, 128, 0) == 2 * 16 * 4096 * 64
+    # V codes are stored in whole 128-token tiles
+    assert L.sa_codes_bytes(2, 16, 4096, 128, 2) == 2 * 16 * 32 * 128 * 64
+    assert L.sa_codes_bytes(1, 1, 416, 64, 2) == 4 * 64 * 64
     assert L.sa_scales_bytes(2, 16, 4096, 128, 0) == 2 * 16 * 32 * 2 * 512
     # ragged N rounds the row tiles up
     assert L.sa_scales_bytes(1, 1, 400, 64, 1) == 4 * 1 * 512
@@ -89,3 +92,23 @@ def test_scales_to_logical_roundtrip():
                 atoms[a * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4] = logical.view(B * H, R, -1)[bh, r, j]
     back = sa.scales_to_logical(atoms, B, H, N, D, "q")
     assert torch.equal(back, logical)
+
+
+def test_v_codes_to_logical_roundtrip():
+    """V codes are stored as 128-token tiles [B,H,ceil(N/128),D,64]; the
+    logical view is [B,H,D,N/2] (channel rows, token pairs)."""
+    import torch
+
+    B, H, N, D = 2, 3, 416, 64
+    NT = (N + 127) // 128
+    logical = torch.randint(0, 256, (B, H, D, N // 2), dtype=torch.uint8)
+    tiled = torch.full((B, H, NT, D, 64), 0xEE, dtype=torch.uint8)  # padding is never read back
+    for t in range(NT):
+        w = min(64, N // 2 - 64 * t)
+        tiled[:, :, t, :, :w] = logical[:, :, :, 64 * t: 64 * t + w]
+    back = sa.codes_to_logical(tiled.reshape(-1), B, H, N, D, "v")
+    assert torch.equal(back, logical)
+    # byte address of (channel d, token n) in the stored layout
+    d, n = 37, 300
+    flat = tiled.reshape(-1)
+    assert flat[((1 * H + 2) * NT + n // 128) * D * 64 + d * 64 + (n % 128) // 2] == logical[1, 2, d, n // 2]

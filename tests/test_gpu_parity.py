@@ -40,7 +40,7 @@ def gpu_quant(x_cpu, role, smooth=True, mode="max"):
 
 def assert_quant_equal(rg, ro, tag=""):
     B, H, N, D = rg.shape
-    codes = rg.codes.cpu().numpy().reshape(ro.codes.shape)
+    codes = sa.codes_to_logical(rg.codes.cpu(), B, H, N, D, rg.role).numpy()
     bad = codes != ro.codes
     assert not bad.any(), f"{tag}: {bad.sum()} code bytes differ, first at {np.argwhere(bad)[:3].tolist()}: " \
                           f"gpu {codes[bad][:8]} oracle {ro.codes[bad][:8]}"
