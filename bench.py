@@ -36,6 +36,17 @@ METRIC = "FP4 attention TOPS (4*B*H*N^2*d, causal halved)"
 L2_FLUSH_BYTES = 256 << 20
 
 
+# DRAM bytes per launch of the dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) on a batch slice of the same
+# workload, scaled by the units of the full launch (traffic grows with the
+# batch: each NVFP4 code and scale byte is read once).  Keyed by workload and
+# kernel; any other pair reports null.
+MEASURED_TRAFFIC = {
+    ("llm", "attn_fwd_pp_kernel<128>"): 14.36e6 * 2,  # B1 slice x 2
+    ("decode", "decode_kernel<128> + combine"): 306.0e6 * 4,  # B8 slice x 4
+}
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -260,6 +271,13 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def traffic_of(w, kname, args):
+    """Measured DRAM bytes per launch for the full workload, else None."""
+    if args.batch is not None or args.mode != "max":
+        return None
+    return MEASURED_TRAFFIC.get((w.name, kname))
+
+
 def config_of(w, mode):
     c = {"workload": w.description, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "causal": w.causal,
          "scale_mode": mode, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
@@ -280,6 +298,8 @@ def main():
     ap.add_argument("--mode", default="max", choices=["max", "search"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (a smaller slice for ncu captures; not a bench line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -287,6 +307,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = wl.WORKLOADS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+
+        w = dataclasses.replace(w, B=args.batch, description=w.description + f" (batch {args.batch} slice)")
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
@@ -377,16 +401,19 @@ def main():
         flops = flops_of(w)
         if w.kind == "decode":
             gbs = hbm_bytes_decode(w) / (ms_attn * 1e-3) / 1e9
-            roof = {"bound": "hbm", "kernel": "decode_kernel<128> + combine", "achieved": gbs, "peak": hbm,
+            kname = "decode_kernel<128> + combine"
+            roof = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm,
                     "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{src} copy bandwidth",
-                    "traffic": None, "ms_per_launch": ms_attn, "algorithmic_bytes": hbm_bytes_decode(w)}
+                    "traffic": traffic_of(w, kname, args), "traffic_unit": "bytes per launch (ncu, batch slice scaled)",
+                    "ms_per_launch": ms_attn, "algorithmic_bytes": hbm_bytes_decode(w)}
         else:
             achieved = flops / (ms_attn * 1e-3) / 1e12
             kname = "attn_fwd_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_pp_kernel<128>"
             roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                     "frac": achieved / fp4_peak,
                     "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
-                    "traffic": None, "ms_per_launch": ms_attn}
+                    "traffic": traffic_of(w, kname, args), "traffic_unit": "bytes per launch (ncu, batch slice scaled)",
+                    "ms_per_launch": ms_attn}
         line = {
             "metric": METRIC, "value": world * flops / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
