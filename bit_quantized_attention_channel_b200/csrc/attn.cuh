@@ -47,7 +47,7 @@ struct AttnParams {
     const float* v_g;
     float* out;
     float* lse;
-    int N, H;
+    int N, H, B;
     int T;    // 128-row tiles of Q/K (= scale row tiles per (b,h))
     int CKv;  // 64-key chunks of the V scale atoms per (b,h)
     int causal;

@@ -31,6 +31,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // 3-D byte tensor {d0 (contiguous), d1, d2}; box {b0, b1, 1}.
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                  uint32_t b1, CUtensorMapSwizzle swz)
 {
@@ -286,6 +299,7 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     p.lse = lse_dev;
     p.N = N;
     p.H = H;
+    p.B = B;
     p.T = sa_cdiv(N, 128);
     p.CKv = sa_cdiv(N, 64);
     p.causal = causal ? 1 : 0;
@@ -318,7 +332,10 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
                 return SA_ERR_CUDA;                                                                         \
             attr_done = 1;                                                                                  \
         }                                                                                                   \
-        attn_fwd_pp_kernel<DD><<<dim3((p.T + 1) / 2, H, B), kPpThreads, smem, stream>>>(tq, tk, tv, p);      \
+        const long nitems = (long)B * H * ((p.T + 1) / 2);                                                \
+        const int nsm = sm_count();                                                                         \
+        if (nsm <= 0) return SA_ERR_CUDA;                                                                   \
+        attn_fwd_pp_kernel<DD><<<(unsigned)(nitems < nsm ? nitems : nsm), kPpThreads, smem, stream>>>(tq, tk, tv, p); \
     } while (0)
     if (D == 128) {
         if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_PP_LAUNCH(128);
