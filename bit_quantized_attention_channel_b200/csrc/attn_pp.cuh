@@ -23,8 +23,12 @@
 //
 // TMEM: one S buffer (128 columns) shared by the two tiles and handed back and
 // forth: Q_A K_u^T -> A loads S -> Q_B K_u^T -> B loads S -> Q_A K_{u+1}^T ...
-// plus O_A, O_B, l_A, l_B and the scale atoms (468 of 512 columns).  Every
-// barrier phase is counted over the CTA's whole item sequence.
+// plus [O_x | l_x] for each tile and the scale factors (472 of 512 columns).
+// The row sum l accumulates the same dequantised P as O: the V operand of
+// P V carries 16 extra rows of E2M1 1.0 (scale 1.0) after row 127, so column
+// 128 of [O_x | l_x] is l (for D = 64, rows 64..127 of the operand are zero).
+// The softmax warps write P's block scales straight into TMEM.  Every barrier
+// phase is counted over the CTA's whole item sequence.
 #pragma once
 
 #include "attn.cuh"
@@ -38,14 +42,11 @@ template <int D>
 struct PpSmem {
     alignas(1024) uint8_t q[2][2][128 * D / 2];  // [item % 2][tile]
     alignas(1024) uint8_t k[kPpStages][128 * D / 2];
-    alignas(1024) uint8_t v[kPpStages][D * 64];
+    alignas(1024) uint8_t v[kPpStages][128 * 64 + 16 * 64];  // V^T (D rows), zero rows to 128, 16 rows of 1.0
     alignas(1024) uint8_t p[2][128 * 64];
-    alignas(1024) uint8_t ones[16 * 64];
     alignas(16) uint8_t qsf[2][2][D / 64 * 512];
     uint8_t ksf[kPpStages][D / 64 * 512];
     uint8_t vsf[kPpStages][2 * 512];
-    uint8_t psf[2][2 * 512];
-    uint8_t onesf[512];
     uint64_t q_full[2];   // [item % 2]: Q tiles and scale atoms landed
     uint64_t q_empty[2];  // [item % 2]: every Q K^T of the item completed
     uint64_t kv_full[kPpStages];
@@ -59,8 +60,10 @@ struct PpSmem {
 };
 
 // TMEM columns
-constexpr uint32_t PP_S = 0, PP_O = 128, PP_L = 384, PP_SFQ = 416, PP_SFK = 432, PP_SFV = 440, PP_SFP = 448,
-                   PP_SF1 = 464;
+// TMEM columns: [O_x | l_x] is PP_OW wide at PP_O + PP_OW x (l in column 128);
+// SFV: 64-key block kb at + 8 kb (V rows in + 0..3, the 1.0 rows' scale at + 4);
+// SFP: tile x at + 8 x, block kb at + 4 kb.
+constexpr uint32_t PP_S = 0, PP_O = 128, PP_OW = 144, PP_SFQ = 416, PP_SFK = 432, PP_SFV = 440, PP_SFP = 456;
 
 SA_DEV bool pp_wait(uint64_t* bar, uint32_t parity, volatile int* abort)
 {
@@ -175,13 +178,28 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    for (int i = tid; i < 16 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.ones)[i] = 0x22222222u;
-    for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
+    // rows D..127 of every V stage are zero, rows 128..143 are E2M1 1.0
+    for (int i = tid; i < kPpStages * (144 - D) * 16; i += blockDim.x) {
+        const int st = i / ((144 - D) * 16), w = i % ((144 - D) * 16);
+        reinterpret_cast<uint32_t*>(s.v[st] + D * 64)[w] = w >= (128 - D) * 16 ? 0x22222222u : 0u;
+    }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = s.tmem_slot;
+    if (warp < 4) {
+        // scale 1.0 for the 1.0 rows of the V operand (B-operand rows 128..143 of
+        // each 64-key block read column base + 4), every lane quadrant
+        const uint32_t one4 = 0x38383838u;
+        for (int kb = 0; kb < 2; kb++)
+            for (int c = 4; c < 8; c++)
+                tmem_st1(tbase + ((uint32_t)(warp * 32) << 16) + PP_SFV + 8 * kb + c, __uint_as_float(one4));
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     if (warp < 4) pp_setmaxnreg_dec<40>();
     if (warp == 0) {
@@ -225,7 +243,6 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            tc_cp_sf(tbase + PP_SF1, smem_u32(s.onesf));
             bool ok = true;
             int g0 = 0;  // ring position of the current item's key tile 0
             int kv_waited = -1, sfk_tile = -1, last_x = -1, last_idx = -1;
@@ -264,22 +281,19 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     last_idx = nS[x]++;
                     return true;
                 };
-                // O_x += P_x V_u, l_x += P_x 1
+                // [O_x | l_x] (+)= P_x [V_u | 0 | 1]
                 auto pv = [&](int x, int u) -> bool {
                     if (!pp_wait(&s.p_full[x], nP[x] & 1, abort)) return false;
                     tc_fence_after();
                     const int nk = min(128, p.N - u * 128);
                     const int kblocks = nk > 64 ? 2 : 1;
-                    for (int kb = 0; kb < kblocks; kb++)
-                        tc_cp_sf(tbase + PP_SFP + 8 * x + 4 * kb, smem_u32(s.psf[x] + 512 * kb));
                     const int st = (g0 + u) % kPpStages;
                     for (int kb = 0; kb < kblocks; kb++) {
                         const uint64_t pd = make_sdesc(smem_u32(s.p[x]) + 32 * kb, 512, 16, 4);
                         const uint32_t acc = (u > 0 || kb > 0) ? 1u : 0u;
-                        mma_fp4(tbase + PP_O + 128 * x, pd, make_sdesc(smem_u32(s.v[st]) + 32 * kb, 512, 16, 4),
-                                idesc_fp4(128, D), tbase + PP_SFP + 8 * x + 4 * kb, tbase + PP_SFV + 4 * kb, acc);
-                        mma_fp4(tbase + PP_L + 16 * x, pd, make_sdesc(smem_u32(s.ones) + 32 * kb, 512, 16, 4),
-                                idesc_fp4(128, 16), tbase + PP_SFP + 8 * x + 4 * kb, tbase + PP_SF1, acc);
+                        mma_fp4(tbase + PP_O + PP_OW * x, pd, make_sdesc(smem_u32(s.v[st]) + 32 * kb, 512, 16, 4),
+                                idesc_fp4(128, PP_OW), tbase + PP_SFP + 8 * x + 4 * kb, tbase + PP_SFV + 8 * kb,
+                                acc);
                     }
                     tc_commit(&s.o_done[x]);
                     nP[x]++;
@@ -296,7 +310,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     const int nk = min(128, p.N - u * 128);
                     const int kblocks = nk > 64 ? 2 : 1;
                     for (int kb = 0; kb < kblocks; kb++)
-                        tc_cp_sf(tbase + PP_SFV + 4 * kb, smem_u32(s.vsf[st] + 512 * kb));
+                        tc_cp_sf(tbase + PP_SFV + 8 * kb, smem_u32(s.vsf[st] + 512 * kb));
                     if (u < I.nuA && !(ok = pv(0, u))) break;
                     if (u + 1 < I.nuB && !(ok = qk(1, u + 1))) break;
                     if (u < I.nuB && !(ok = pv(1, u))) break;
@@ -392,11 +406,12 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     *reinterpret_cast<uint4*>(prow + cs * 16) =
                         make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
                 }
-                *reinterpret_cast<uint32_t*>(s.psf[x] + (r & 31) * 16 + (r >> 5) * 4) = scw0;
-                *reinterpret_cast<uint32_t*>(s.psf[x] + 512 + (r & 31) * 16 + (r >> 5) * 4) = scw1;
+                // P's block scales into TMEM: row r reads (lane r, column base + r / 32)
+                tmem_st1(tbase + lane_off + PP_SFP + 8 * x + quad, __uint_as_float(scw0));
+                tmem_st1(tbase + lane_off + PP_SFP + 8 * x + 4 + quad, __uint_as_float(scw1));
                 if (u > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
                     // rescale this row of O (64 columns per round trip) and l
-                    const uint32_t oa = tbase + lane_off + PP_O + 128 * x;
+                    const uint32_t oa = tbase + lane_off + PP_O + PP_OW * x;
 #pragma unroll
                     for (int h = 0; h < D / 64; h++) {
                         float o0[32], o1[32];
@@ -413,10 +428,10 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                         tmem_st32(oa + 64 * h, o0);
                         tmem_st32(oa + 64 * h + 32, o1);
                     }
-                    const float lv = tmem_ld1_sync(tbase + lane_off + PP_L + 16 * x);
-                    tmem_st1(tbase + lane_off + PP_L + 16 * x, lv * alpha);
-                    tmem_wait_st();
+                    const float lv = tmem_ld1_sync(oa + 128);
+                    tmem_st1(oa + 128, lv * alpha);
                 }
+                tmem_wait_st();
                 fence_proxy_async();
                 tc_fence_before();
                 __syncwarp();
@@ -429,13 +444,13 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 break;
             }
             tc_fence_after();
-            const float l = tmem_ld1_sync(tbase + lane_off + PP_L + 16 * x);
+            const float l = tmem_ld1_sync(tbase + lane_off + PP_O + PP_OW * x + 128);
             const float scale = p.v_g[0] / l;
             float* orow = p.out + ((size_t)I.bh * p.N + row) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; c++) {
                 float o[32];
-                tmem_ld32(tbase + lane_off + PP_O + 128 * x + 32 * c, o);
+                tmem_ld32(tbase + lane_off + PP_O + PP_OW * x + 32 * c, o);
                 tmem_wait_ld();
                 reg_fence(o);
                 if (row < p.N) {
