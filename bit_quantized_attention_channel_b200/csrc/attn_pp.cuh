@@ -47,6 +47,7 @@ struct PpSmem {
     alignas(16) uint8_t qsf[2][2][D / 64 * 512];
     uint8_t ksf[kPpStages][D / 64 * 512];
     uint8_t vsf[kPpStages][2 * 512];
+    float lg2tab[16];  // log2 of E4M3 significands: [m] normal (1 + m/8), [8 + m] subnormal (m/4)
     uint64_t q_full[2];   // [item % 2]: Q tiles and scale atoms landed
     uint64_t q_empty[2];  // [item % 2]: every Q K^T of the item completed
     uint64_t kv_full[kPpStages];
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
+    if (tid < 16) s.lg2tab[tid] = tid < 8 ? log2f(1.0f + tid * 0.125f) : log2f((tid - 8) * 0.25f);
     // rows D..127 of every V stage are zero, rows 128..143 are E2M1 1.0
     for (int i = tid; i < kPpStages * (144 - D) * 16; i += blockDim.x) {
         const int st = i / ((144 - D) * 16), w = i % ((144 - D) * 16);
@@ -375,22 +377,32 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 const float msub = m2_new == -INFINITY ? 0.0f : m2_new;
                 const float alpha = ex2f(m2 - msub);
                 m2 = m2_new;
-                uint32_t codes[16];
+                // block scales first (eight independent chains): E4M3 of (block max of
+                // P * 2688) / 6, and log2 of the scale value from the exponent and a
+                // table of significands
+                const float lm = kLog2_2688 - msub;
+                float bias[8];
                 uint32_t scw0 = 0, scw1 = 0;
 #pragma unroll
                 for (int blk = 0; blk < 8; blk++) {
-                    const float pmax = ex2f(fmaf(bmax[blk], c2, kLog2_2688 - msub));
-                    const uint32_t sc = f32_to_e4m3(pmax * (1.0f / 6.0f));
-                    const float bias = sc ? (kLog2_2688 - msub - lg2f(e4m3_to_f32(sc))) : -INFINITY;
-                    float y[16];
-#pragma unroll
-                    for (int i2 = 0; i2 < 16; i2++) y[i2] = ex2f(fmaf(sv[16 * blk + i2], c2, bias));
-                    codes[2 * blk] = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-                    codes[2 * blk + 1] = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+                    const uint32_t sc = f32_to_e4m3(ex2f(fmaf(bmax[blk], c2, lm)) * (1.0f / 6.0f));
+                    const uint32_t e = sc >> 3, m = sc & 7u;
+                    const float lg2s = (e ? (float)((int)e - 7) : -7.0f) + s.lg2tab[(e ? 0u : 8u) + m];
+                    bias[blk] = sc ? lm - lg2s : -INFINITY;
                     if (blk < 4)
                         scw0 |= sc << (8 * blk);
                     else
                         scw1 |= sc << (8 * (blk - 4));
+                }
+                // y = P * 2688 / scale, rounded to E2M1
+                uint32_t codes[16];
+#pragma unroll
+                for (int blk = 0; blk < 8; blk++) {
+                    float y[16];
+#pragma unroll
+                    for (int i2 = 0; i2 < 16; i2++) y[i2] = ex2f(fmaf(sv[16 * blk + i2], c2, bias[blk]));
+                    codes[2 * blk] = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+                    codes[2 * blk + 1] = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
                 }
                 // P buffer and O are free once this role's previous P V finished
                 // (for u = 0 that is the previous item's last one)
