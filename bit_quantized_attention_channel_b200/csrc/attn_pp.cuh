@@ -35,7 +35,7 @@
 
 namespace sa {
 
-constexpr int kPpStages = 3;
+constexpr int kPpStages = 4;
 constexpr int kPpThreads = 384;
 
 template <int D>
@@ -458,18 +458,40 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             tc_fence_after();
             const float l = tmem_ld1_sync(tbase + lane_off + PP_O + PP_OW * x + 128);
             const float scale = p.v_g[0] / l;
-            float* orow = p.out + ((size_t)I.bh * p.N + row) * D;
+            {
+                // Stage 32 rows x 16 floats of O per round in this warp's 2 KB of the
+                // tile's P buffer (idle until the next item's first P), 16-byte units
+                // XOR-swizzled by row / 2, then write 64-byte row segments: each store
+                // instruction covers 8 rows.
+                float4* stage = reinterpret_cast<float4*>(s.p[x] + quad * 2048);
+                const int row0 = tq * 128 + quad * 32;
+                float* obase = p.out + ((size_t)I.bh * p.N + row0) * D;
+#pragma unroll 1
+                for (int c = 0; c < D / 16; c++) {
+                    uint32_t o[16];
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+                        "%12, %13, %14, %15}, [%16];\n\t"
+                        "tcgen05.wait::ld.sync.aligned;"
+                        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]),
+                          "=r"(o[7]), "=r"(o[8]), "=r"(o[9]), "=r"(o[10]), "=r"(o[11]), "=r"(o[12]), "=r"(o[13]),
+                          "=r"(o[14]), "=r"(o[15])
+                        : "r"(tbase + lane_off + PP_O + PP_OW * x + 16 * c)
+                        : "memory");
 #pragma unroll
-            for (int c = 0; c < D / 32; c++) {
-                float o[32];
-                tmem_ld32(tbase + lane_off + PP_O + PP_OW * x + 32 * c, o);
-                tmem_wait_ld();
-                reg_fence(o);
-                if (row < p.N) {
+                    for (int j2 = 0; j2 < 4; j2++)
+                        stage[lane * 4 + (j2 ^ ((lane >> 1) & 3))] =
+                            make_float4(__uint_as_float(o[4 * j2]) * scale, __uint_as_float(o[4 * j2 + 1]) * scale,
+                                        __uint_as_float(o[4 * j2 + 2]) * scale, __uint_as_float(o[4 * j2 + 3]) * scale);
+                    __syncwarp();
 #pragma unroll
-                    for (int i2 = 0; i2 < 32; i2 += 4)
-                        *reinterpret_cast<float4*>(orow + 32 * c + i2) =
-                            make_float4(o[i2] * scale, o[i2 + 1] * scale, o[i2 + 2] * scale, o[i2 + 3] * scale);
+                    for (int i2 = 0; i2 < 4; i2++) {
+                        const int rr = 8 * i2 + (lane >> 2), jj = lane & 3;
+                        if (row0 + rr < p.N)
+                            *reinterpret_cast<float4*>(obase + (size_t)rr * D + 16 * c + 4 * jj) =
+                                stage[rr * 4 + (jj ^ ((rr >> 1) & 3))];
+                    }
+                    __syncwarp();
                 }
             }
             if (p.lse && row < p.N) p.lse[(size_t)I.bh * p.N + row] = m2 * kLn2 + logf(l * (1.0f / 2688.0f));
