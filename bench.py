@@ -152,9 +152,9 @@ class Path:
         w, st = self.w, self.st
         if w.kind == "decode":
             return  # the KV cache is quantised once, before timing (it is a cache)
-        st["q"] = sa.sa_quant_nvfp4(self.q, "q", mode=self.mode, out=st.get("q"))
-        st["k"] = sa.sa_quant_nvfp4(self.k, "k", mode=self.mode, out=st.get("k"))
-        st["v"] = sa.sa_quant_nvfp4(self.v, "v", mode=self.mode, out=st.get("v"))
+        # Q, K (smoothed) and V in two launches: statistics, then quantisation
+        st["qkv"] = sa.sa_quant_nvfp4_qkv(self.q, self.k, self.v, smooth=True, mode=self.mode, out=st.get("qkv"))
+        st["q"], st["k"], st["v"] = st["qkv"]
         if w.thrift_bp:
             st["mask"], _ = sa.sa_thrift_select(self.q, self.k, w.causal, w.thrift_bp)
 
@@ -201,7 +201,7 @@ class Path:
 def kernels_per_step(w):
     if w.kind == "decode":
         return 3  # q amax, split kernel, combine
-    n = 2 + 3 + 2 + 1  # q: amax+quant, k: stats+final+quant, v: amax+quant, attention
+    n = 2 + 1  # fused pre-pass: statistics + quantisation of Q, K, V; attention
     if w.thrift_bp:
         n += 3  # pool, score, top-k
     return n

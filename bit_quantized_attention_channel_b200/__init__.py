@@ -8,6 +8,7 @@ raised.
 
 Entry points keep the C names:
   sa_quant_nvfp4        smoothing + NVFP4 pre-pass (max-scaling or ScaleSearch)
+  sa_quant_nvfp4_qkv    the same for Q, K and V of one shape in two launches
   sa_thrift_select      high-precision block selector
   sa_attn_fwd           NVFP4 attention forward (optionally with bf16 blocks)
   sa_attn_decode_kvfp4  decode over an NVFP4 KV cache
@@ -55,6 +56,9 @@ def lib():
         L.sa_quant_nvfp4.restype = I
         L.sa_quant_nvfp4_noalloc.argtypes = [P, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P]
         L.sa_quant_nvfp4_noalloc.restype = I
+        L.sa_quant_qkv_workspace_size.argtypes, L.sa_quant_qkv_workspace_size.restype = [I, I, I, I], Z
+        L.sa_quant_nvfp4_qkv.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, Z, P]
+        L.sa_quant_nvfp4_qkv.restype = I
         L.sa_select_workspace_size.argtypes, L.sa_select_workspace_size.restype = [I, I, I, I], Z
         L.sa_thrift_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P, Z, P]
         L.sa_thrift_select.restype = I
@@ -131,6 +135,36 @@ def sa_quant_nvfp4(x, role: str, smooth: bool = True, mode: str = "max", f_lo: i
                             _ptr(out.scales), _ptr(out.g), _ptr(out.k_mean), _ptr(out.ss_off), _ptr(ws), ws_bytes,
                             _stream(stream)))
     return out
+
+
+def sa_quant_nvfp4_qkv(q, k, v, smooth: bool = True, mode: str = "max", f_lo: int = -2, f_hi: int = 6,
+                       out=None, stream=None):
+    """Pre-pass of Q, K (smoothed when `smooth`) and V of one shape in two
+    launches; same results as three sa_quant_nvfp4 calls.  Returns
+    (NVFP4Tensor q, k, v); `out` may pass the three to reuse."""
+    import torch
+
+    B, H, N, D = q.shape
+    for t in (q, k, v):
+        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and tuple(t.shape) == (B, H, N, D)
+    L = lib()
+    if out is None:
+        out = []
+        for role, r in (("q", 0), ("k", 1), ("v", 2)):
+            codes = _empty(L.sa_codes_bytes(B, H, N, D, r), q.device)
+            scales = _empty(L.sa_scales_bytes(B, H, N, D, r), q.device)
+            g = torch.empty(2, dtype=torch.float32, device=q.device)
+            km = torch.empty(B, H, D, dtype=torch.float32, device=q.device) if (role == "k" and smooth) else None
+            out.append(NVFP4Tensor(codes, scales, g, role, (B, H, N, D), km, None))
+    qt, kt, vt = out
+    ws_bytes = L.sa_quant_qkv_workspace_size(B, H, N, D)
+    ws = _empty(ws_bytes, q.device)
+    _check("sa_quant_nvfp4_qkv",
+           L.sa_quant_nvfp4_qkv(_ptr(q), _ptr(k), _ptr(v), B, H, N, D, int(smooth), SA_SCALE[mode], f_lo, f_hi,
+                                _ptr(qt.codes), _ptr(qt.scales), _ptr(qt.g), _ptr(kt.codes), _ptr(kt.scales),
+                                _ptr(kt.g), _ptr(kt.k_mean), _ptr(vt.codes), _ptr(vt.scales), _ptr(vt.g), _ptr(ws),
+                                ws_bytes, _stream(stream)))
+    return qt, kt, vt
 
 
 def sa_thrift_select(q, k, causal: bool, frac_bp: int = 500, stream=None):

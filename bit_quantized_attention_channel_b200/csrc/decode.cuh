@@ -39,6 +39,7 @@ struct DecSmem {
     alignas(16) uint8_t qsf[D / 64 * 512];
     uint8_t psf[2 * 512];
     uint8_t onesf[512];
+    float rcp[128];  // reciprocals of the E4M3 scale values
     float red[4][kDecN];
     float mnew[kDecN];
     float alpha[kDecN];
@@ -77,6 +78,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     {
         float g, inv_g;
         tensor_scale(__uint_as_float(*p.q_amax), g, inv_g);
+        fill_rcp_table(s.rcp);
         for (int e = tid; e < kDecN * D / 2; e += blockDim.x) s.q[e] = 0;
         for (int e = tid; e < KB * 512; e += blockDim.x) s.qsf[e] = 0;
         __syncthreads();
@@ -89,7 +91,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
             for (int i = 0; i < 16; i++) xt[i] = __fmul_rn(bf16_bits_to_f32(src[i]), inv_g);
             uint32_t c0, c1, sc;
             int off;
-            quant16<false>(xt, 0, 1, c0, c1, sc, off);
+            quant16<false>(xt, 0, 1, c0, c1, sc, off, s.rcp);
             // row hi, bytes 8j..8j+7 of a (D/2)-byte row, swizzled in 16-byte chunks
             const int byte = 8 * j;
             const int chunk = byte >> 4;

@@ -28,18 +28,48 @@ constexpr int kTile = 128;
 // Block quantisation (device)
 // ---------------------------------------------------------------------------
 
+// x / 6 rounded to nearest even.  For x >= 2^-120 the product by RN(1/6)
+// corrected by one FMA residual step equals the IEEE quotient (checked
+// exhaustively over every float in that range); smaller x divide directly.
+SA_DEV float div6_rn(float x)
+{
+    if (x < 7.52316384526264e-37f) return __fdiv_rn(x, 6.0f);  // 2^-120
+    const float r6 = 0.16666667163372040f;                    // RN(1/6)
+    const float q0 = __fmul_rn(x, r6);
+    return __fmaf_rn(__fmaf_rn(-q0, 6.0f, x), r6, q0);
+}
+
+// Exact reciprocals of the 127 nonzero E4M3 scale values (IEEE RN), one
+// table per CTA in shared memory.
+SA_DEV void fill_rcp_table(float* rcp)
+{
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) rcp[c] = c ? __frcp_rn(e4m3_to_f32((uint32_t)c)) : 0.0f;
+}
+
+// Two products a_i * b in one instruction (IEEE RN per lane).
+SA_DEV void mul2_rn(float a0, float a1, float b, float& r0, float& r1)
+{
+    asm("{\n\t.reg .b64 a, bb, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 bb, {%4, %4};\n\t"
+        "mul.rn.f32x2 d, a, bb;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b));
+}
+
 // Codes of 16 g-normalised values for scale byte c: r = 1/s (IEEE),
 // y = x~ * r (IEEE), E2M1 round-to-nearest-even.  c == 0 -> all zero.
-SA_DEV void encode16(const float (&xt)[16], uint32_t c, uint32_t& w0, uint32_t& w1)
+SA_DEV void encode16(const float (&xt)[16], uint32_t c, uint32_t& w0, uint32_t& w1, const float* rcp)
 {
     if (c == 0) {
         w0 = w1 = 0;
         return;
     }
-    float r = __frcp_rn(e4m3_to_f32(c));
+    const float r = rcp[c];
     float y[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++) y[i] = __fmul_rn(xt[i], r);
+    for (int i = 0; i < 16; i += 2) mul2_rn(xt[i], xt[i + 1], r, y[i], y[i + 1]);
     w0 = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
     w1 = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
 }
@@ -66,13 +96,15 @@ SA_DEV float err16(const float (&xt)[16], uint32_t c, uint32_t w0, uint32_t w1)
 // f in [f_lo, f_hi) \ {0} are tried in ascending order and replace the best
 // only when strictly better (f = 0 wins ties, then the lowest f).
 template <bool SEARCH>
-SA_DEV void quant16(const float (&xt)[16], int f_lo, int f_hi, uint32_t& w0, uint32_t& w1, uint32_t& sc, int& off)
+SA_DEV void quant16(const float (&xt)[16], int f_lo, int f_hi, uint32_t& w0, uint32_t& w1, uint32_t& sc, int& off,
+                    const float* rcp)
 {
-    float amax = 0.0f;
+    float a[8];
 #pragma unroll
-    for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(xt[i]));
-    uint32_t c0 = f32_to_e4m3(__fdiv_rn(amax, 6.0f));
-    encode16(xt, c0, w0, w1);
+    for (int i = 0; i < 8; i++) a[i] = fmaxf(fabsf(xt[2 * i]), fabsf(xt[2 * i + 1]));
+    const float amax = fmaxf(fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])), fmaxf(fmaxf(a[4], a[5]), fmaxf(a[6], a[7])));
+    uint32_t c0 = f32_to_e4m3(div6_rn(amax));
+    encode16(xt, c0, w0, w1, rcp);
     sc = c0;
     off = 0;
     if (SEARCH && c0 != 0) {
@@ -81,7 +113,7 @@ SA_DEV void quant16(const float (&xt)[16], int f_lo, int f_hi, uint32_t& w0, uin
             int c = (int)c0 + f;
             if (f == 0 || c < 0 || c > 0x7E) continue;
             uint32_t t0, t1;
-            encode16(xt, (uint32_t)c, t0, t1);
+            encode16(xt, (uint32_t)c, t0, t1, rcp);
             float e = err16(xt, (uint32_t)c, t0, t1);
             if (e < best) {
                 best = e;
@@ -139,32 +171,26 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const uint4* __restrict_
     }
 }
 
-// K statistics per (b,h, 128-token tile): each thread owns a channel pair and
-// walks the tile's tokens in ascending order (FP64 sum, FP32 max/min).
+// K statistics of one (b,h, 128-token tile, channel pair): tokens in ascending
+// order (FP64 sum, FP32 max/min).  Returns false on a non-finite value.
 template <int D>
-__global__ void __launch_bounds__(256) kstats_kernel(const uint32_t* __restrict__ x, int N, int T,
-                                                     double* __restrict__ psum, float* __restrict__ pmax,
-                                                     float* __restrict__ pmin)
+SA_DEV bool kstats_pair(const uint32_t* __restrict__ x, int N, int T, size_t bh, int tile, int cp,
+                        double* __restrict__ psum, float* __restrict__ pmax, float* __restrict__ pmin)
 {
-    constexpr int P = D / 2;       // channel pairs per row
-    constexpr int TPB = 256 / P;   // tiles per block
-    int cp = threadIdx.x % P;
-    int tile = blockIdx.x * TPB + threadIdx.x / P;
-    size_t bh = blockIdx.y;
-    if (tile >= T) return;
-    int r0 = tile * kTile;
-    int rows = min(kTile, N - r0);
+    constexpr int P = D / 2;  // channel pairs per row
+    const int r0 = tile * kTile;
+    const int rows = min(kTile, N - r0);
     const uint32_t* p = x + (bh * N + r0) * P + cp;
     double s0 = 0.0, s1 = 0.0;
     float mx0 = -INFINITY, mx1 = -INFINITY, mn0 = INFINITY, mn1 = INFINITY;
     bool bad = false;
-    for (int r0b = 0; r0b < rows; r0b += 16) {
-        uint32_t w[16];
+    for (int r0b = 0; r0b < rows; r0b += 32) {
+        uint32_t w[32];
 #pragma unroll
-        for (int u = 0; u < 16; u++) w[u] = r0b + u < rows ? __ldcs(p + (size_t)(r0b + u) * P) : 0u;
-        const int nr = min(16, rows - r0b);
+        for (int u = 0; u < 32; u++) w[u] = r0b + u < rows ? __ldg(p + (size_t)(r0b + u) * P) : 0u;
+        const int nr = min(32, rows - r0b);
 #pragma unroll
-        for (int u = 0; u < 16; u++) {
+        for (int u = 0; u < 32; u++) {
             if (u >= nr) break;
             float a = bf16_bits_to_f32(w[u] & 0xFFFFu), b = bf16_bits_to_f32(w[u] >> 16);
             bad |= !isfinite(a) || !isfinite(b);
@@ -176,52 +202,71 @@ __global__ void __launch_bounds__(256) kstats_kernel(const uint32_t* __restrict_
             mn1 = fminf(mn1, b);
         }
     }
-    if (bad) sa_raise(SA_ERR_NONFINITE);
-    size_t o = (bh * T + tile) * D + 2 * cp;
+    const size_t o = (bh * T + tile) * D + 2 * cp;
     psum[o] = s0;
     psum[o + 1] = s1;
     pmax[o] = mx0;
     pmax[o + 1] = mx1;
     pmin[o] = mn0;
     pmin[o + 1] = mn1;
+    return !bad;
+}
+
+// K statistics per (b,h, 128-token tile): each thread owns a channel pair and
+// walks the tile's tokens in ascending order (FP64 sum, FP32 max/min).
+template <int D>
+__global__ void __launch_bounds__(256) kstats_kernel(const uint32_t* __restrict__ x, int N, int T,
+                                                     double* __restrict__ psum, float* __restrict__ pmax,
+                                                     float* __restrict__ pmin)
+{
+    constexpr int P = D / 2;       // channel pairs per row
+    constexpr int TPB = 256 / P;   // tiles per block
+    const int cp = threadIdx.x % P;
+    const int tile = blockIdx.x * TPB + threadIdx.x / P;
+    if (tile >= T) return;
+    if (!kstats_pair<D>(x, N, T, blockIdx.y, tile, cp, psum, pmax, pmin)) sa_raise(SA_ERR_NONFINITE);
 }
 
 // Per (b,h,channel): sum the tile partials in tile order, mean = FP32(sum/N);
-// amax contribution max(fl(max - mean), fl(mean - min)).
+// returns the amax contribution max(fl(max - mean), fl(mean - min)), >= 0.
+// Partials are read through L2 (they may come from other CTAs of this grid).
+SA_DEV float kfinal_channel(const double* __restrict__ psum, const float* __restrict__ pmax,
+                            const float* __restrict__ pmin, int N, int T, int D, size_t bh, int c,
+                            float* __restrict__ kmean)
+{
+    double total = 0.0;
+    float mx = -INFINITY, mn = INFINITY;
+    for (int t0 = 0; t0 < T; t0 += 8) {
+        double ps[8];
+        float px[8], pn[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            const size_t o = (bh * T + min(t0 + u, T - 1)) * D + c;
+            ps[u] = __ldcg(psum + o);
+            px[u] = __ldcg(pmax + o);
+            pn[u] = __ldcg(pmin + o);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            if (t0 + u >= T) break;
+            total = __dadd_rn(total, ps[u]);  // tiles in ascending order
+            mx = fmaxf(mx, px[u]);
+            mn = fminf(mn, pn[u]);
+        }
+    }
+    const float mu = __double2float_rn(__ddiv_rn(total, (double)N));
+    kmean[bh * D + c] = mu;
+    return fmaxf(fmaxf(__fsub_rn(mx, mu), __fsub_rn(mu, mn)), 0.0f);
+}
+
 __global__ void __launch_bounds__(128) kfinal_kernel(const double* __restrict__ psum,
                                                      const float* __restrict__ pmax,
                                                      const float* __restrict__ pmin, int N, int T, int D,
                                                      float* __restrict__ kmean, unsigned* __restrict__ amax_word)
 {
-    size_t bh = blockIdx.x;
-    int c = threadIdx.x;
-    float a = 0.0f;
-    if (c < D) {
-        double total = 0.0;
-        float mx = -INFINITY, mn = INFINITY;
-        for (int t0 = 0; t0 < T; t0 += 8) {
-            double ps[8];
-            float px[8], pn[8];
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                const size_t o = (bh * T + min(t0 + u, T - 1)) * D + c;
-                ps[u] = psum[o];
-                px[u] = pmax[o];
-                pn[u] = pmin[o];
-            }
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                if (t0 + u >= T) break;
-                total = __dadd_rn(total, ps[u]);  // tiles in ascending order
-                mx = fmaxf(mx, px[u]);
-                mn = fminf(mn, pn[u]);
-            }
-        }
-        float mu = __double2float_rn(__ddiv_rn(total, (double)N));
-        kmean[bh * D + c] = mu;
-        a = fmaxf(__fsub_rn(mx, mu), __fsub_rn(mu, mn));
-        a = fmaxf(a, 0.0f);
-    }
+    const size_t bh = blockIdx.x;
+    const int c = threadIdx.x;
+    float a = c < D ? kfinal_channel(psum, pmax, pmin, N, T, D, bh, c, kmean) : 0.0f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     if ((threadIdx.x & 31) == 0) atomicMax(amax_word, __float_as_uint(a));
@@ -231,98 +276,352 @@ __global__ void __launch_bounds__(128) kfinal_kernel(const double* __restrict__ 
 // Quantisation kernels
 // ---------------------------------------------------------------------------
 
-// Q/K: thread per 16-channel block.  nblk = B*H*N*(D/16).
+// ---------------------------------------------------------------------------
+// Tile quantisers: one CTA per (b,h, 128-row tile) of Q/K or (b,h, 128-token
+// tile) of V.  Loads are 16-byte and coalesced; each thread encodes the four
+// blocks of one 64-element chunk, writes their codes as one contiguous 32-byte
+// piece, and assembles the four scale bytes as one word of the tile's scale
+// atoms in shared memory; the atoms (padding zero) go out as 16-byte stores.
+// Per block the arithmetic is quant16, so the bytes equal the per-block
+// kernels'.
+// ---------------------------------------------------------------------------
+
+// Q/K tile: 128 rows x D channels; thread t -> row t / (D/64), chunk t % (D/64).
+// The tile is staged in shared memory by coalesced 16-byte loads (all issued
+// before the first store).  16-byte piece c of row r sits at piece
+// (c & ~7) | ((c ^ (r * CK + c / 8)) & 7) of that row, so that the eight
+// threads of a shared-memory phase (eight different (row, chunk) pairs) read
+// eight different bank groups.
 template <int D, bool SMOOTH, bool SEARCH>
-__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ x, size_t nblk, int N, int RT,
-                                                         const float* __restrict__ kmean,
-                                                         const unsigned* __restrict__ amax_word, int f_lo,
-                                                         int f_hi, uint2* __restrict__ codes,
-                                                         uint8_t* __restrict__ scales,
-                                                         int8_t* __restrict__ ss_off, float* __restrict__ g_out)
+SA_DEV void quant_rows_tile(const uint4* __restrict__ x, size_t bh, int tile, int N, const float* __restrict__ kmean,
+                            float inv_g, int f_lo, int f_hi, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                            int8_t* __restrict__ ss_off, uint4* xs /* shared, 128 * D / 8 */,
+                            uint32_t* atoms /* shared, CK * 128 words */, const float* rcp /* shared, filled */)
 {
-    constexpr int NB = D / 16, CK = D / 64;
-    float g, inv_g;
-    tensor_scale(__uint_as_float(*amax_word), g, inv_g);
-    size_t stride = (size_t)gridDim.x * blockDim.x;
-    size_t b0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (b0 == 0) {
-        g_out[0] = g;
-        g_out[1] = inv_g;
-    }
-    for (size_t b = b0; b < nblk; b += stride) {
-        size_t row = b / NB;
-        int j = (int)(b % NB);
-        size_t bh = row / N;
-        int n = (int)(row % N);
-        uint4 u0 = __ldcs(x + 2 * b), u1 = __ldcs(x + 2 * b + 1);
-        uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        float xt[16];
+    constexpr int CK = D / 64, NB = D / 16, RP = D / 8;  // 16-byte pieces per row
+    constexpr int NTH = 128 * CK, PER = 128 * RP / NTH;  // threads, pieces per thread
+    const int t = threadIdx.x;
+    const int r = t / CK, ck = t % CK;
+    const int n = tile * 128 + r;
+    const int T = (N + 127) / 128;
+    const int rows = min(128, N - tile * 128);
+    {
+        const uint4* src = x + (bh * N + (size_t)tile * 128) * RP;
+        uint4 u[PER];
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            float v = bf16_bits_to_f32((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
-            if (SMOOTH) v = __fsub_rn(v, __ldg(kmean + bh * D + j * 16 + i));
-            xt[i] = __fmul_rn(v, inv_g);
+        for (int k = 0; k < PER; k++) {
+            const int i = t + k * NTH;
+            u[k] = i < rows * RP ? __ldcs(src + i) : make_uint4(0, 0, 0, 0);
         }
-        uint32_t c0, c1, sc;
-        int off;
-        quant16<SEARCH>(xt, f_lo, f_hi, c0, c1, sc, off);
-        codes[b] = make_uint2(c0, c1);
-        size_t atom = (bh * RT + (size_t)(n >> 7)) * CK + (size_t)(j >> 2);
-        scales[atom * 512 + sf_atom_offset((uint32_t)(n & 127), (uint32_t)(j & 3))] = (uint8_t)sc;
-        if (ss_off) ss_off[b] = (int8_t)off;
+#pragma unroll
+        for (int k = 0; k < PER; k++) {
+            const int i = t + k * NTH, rr = i / RP, c = i % RP;
+            xs[rr * RP + ((c & ~7) | ((c ^ (rr * CK + c / 8)) & 7))] = u[k];
+        }
+    }
+    for (int i = t; i < CK * 128; i += blockDim.x) atoms[i] = 0u;
+    __syncthreads();
+    if (n < N) {
+        const size_t row = bh * N + n;
+        uint32_t word = 0;
+        uint2 cw[4];
+        uint32_t offw = 0;
+#pragma unroll
+        for (int jb = 0; jb < 4; jb++) {
+            uint4 ua, ub;
+            {
+                const int c0 = ck * 8 + 2 * jb, c1 = c0 + 1;
+                ua = xs[r * RP + ((c0 & ~7) | ((c0 ^ (r * CK + ck)) & 7))];
+                ub = xs[r * RP + ((c1 & ~7) | ((c1 ^ (r * CK + ck)) & 7))];
+            }
+            const uint32_t w[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+            const int j = ck * 4 + jb;
+            float xt[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                float v0 = __uint_as_float(w[i >> 1] << 16), v1 = __uint_as_float(w[i >> 1] & 0xFFFF0000u);
+                if (SMOOTH) {
+                    v0 = __fsub_rn(v0, __ldg(kmean + bh * D + j * 16 + i));
+                    v1 = __fsub_rn(v1, __ldg(kmean + bh * D + j * 16 + i + 1));
+                }
+                mul2_rn(v0, v1, inv_g, xt[i], xt[i + 1]);
+            }
+            uint32_t c0, c1, sc;
+            int off;
+            quant16<SEARCH>(xt, f_lo, f_hi, c0, c1, sc, off, rcp);
+            cw[jb] = make_uint2(c0, c1);
+            word |= sc << (8 * jb);
+            offw |= ((uint32_t)(uint8_t)(int8_t)off) << (8 * jb);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(codes + row * NB + ck * 4);
+        dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+        dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+        atoms[ck * 128 + (r & 31) * 4 + (r >> 5)] = word;
+        if (ss_off) *reinterpret_cast<uint32_t*>(ss_off + row * NB + ck * 4) = offw;
+    }
+    __syncthreads();
+    // atom (bh, tile, ck): 512 bytes = 32 x uint4
+    for (int i = t; i < CK * 32; i += blockDim.x) {
+        const int ck2 = i / 32, q = i % 32;
+        const uint32_t* a = atoms + ck2 * 128 + q * 4;
+        reinterpret_cast<uint4*>(scales + (((size_t)bh * T + tile) * CK + ck2) * 512)[q] = make_uint4(a[0], a[1], a[2], a[3]);
     }
 }
 
-// V: thread per (4 channels, 16-token block); codes land in 128-token tiles
-// [B,H,ceil(N/128),D,64] (each tile's V^T block is one contiguous D x 64-byte
-// region, the operand of one P V MMA).
-// nblk4 = B*H*(N/16)*(D/4), channel group fastest so a warp reads 256
-// contiguous bytes of each token row.
+// V tile: tokens 128 tile .. +127 x D channels, staged in shared memory
+// (row-major bf16, 128 x D); thread t -> channel t % D, token half t / D
+// (blocks 4 half .. 4 half + 3 of the tile).
 template <bool SEARCH>
-__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ x, size_t nblk4, int N, int D,
+SA_DEV void quant_v_tile(const uint16_t* __restrict__ x, size_t bh, int tile, int N, int D, float inv_g, int f_lo,
+                         int f_hi, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                         int8_t* __restrict__ ss_off, uint16_t* xs /* shared, 128 * D */,
+                         uint32_t* atoms /* shared, 2 * 128 words */, const float* rcp /* shared, filled */)
+{
+    const int t = threadIdx.x;
+    const int NT = (N + 127) / 128, CK = (N + 63) / 64, NBT = N / 16;
+    const int rows = min(128, N - tile * 128);
+    // coalesced 16-byte loads of the tile
+    const uint4* src = reinterpret_cast<const uint4*>(x + (bh * N + (size_t)tile * 128) * D);
+    for (int i = t; i < rows * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(xs)[i] = __ldcs(src + i);
+    for (int i = t; i < 256; i += blockDim.x) atoms[i] = 0u;
+    __syncthreads();
+    const int c = t % D, half = t / D;
+    if (half < 2) {
+        uint32_t word = 0, offw = 0;
+        uint2 cw[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
+#pragma unroll
+        for (int jb = 0; jb < 4; jb++) {
+            const int tok0 = half * 64 + jb * 16;
+            if (tok0 >= rows) break;
+            float xt[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+                mul2_rn(bf16_bits_to_f32(xs[(tok0 + i) * D + c]), bf16_bits_to_f32(xs[(tok0 + i + 1) * D + c]), inv_g,
+                        xt[i], xt[i + 1]);
+            uint32_t q0, q1, sc;
+            int off;
+            quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off, rcp);
+            cw[jb] = make_uint2(q0, q1);
+            word |= sc << (8 * jb);
+            offw |= ((uint32_t)(uint8_t)(int8_t)off) << (8 * jb);
+        }
+        const int nblk_here = min(4, max(0, (rows - half * 64) / 16));
+        if (nblk_here > 0) {
+            uint8_t* dst = codes + (((size_t)bh * NT + tile) * D + c) * 64 + half * 32;
+            if (nblk_here == 4) {
+                reinterpret_cast<uint4*>(dst)[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+                reinterpret_cast<uint4*>(dst)[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+            } else {
+                for (int jb = 0; jb < nblk_here; jb++) reinterpret_cast<uint2*>(dst)[jb] = cw[jb];
+            }
+            atoms[half * 128 + (c & 31) * 4 + ((c & 127) >> 5)] = word;
+            if (ss_off) {
+                int8_t* so = ss_off + ((size_t)bh * D + c) * NBT + tile * 8 + half * 4;
+                for (int jb = 0; jb < nblk_here; jb++) so[jb] = (int8_t)(offw >> (8 * jb));
+            }
+        }
+    }
+    __syncthreads();
+    // atoms (bh, channel tile 0, chunks 2 tile, 2 tile + 1), only chunks inside N
+    for (int i = t; i < 64; i += blockDim.x) {
+        const int h2 = i / 32, q = i % 32;
+        const int ck = 2 * tile + h2;
+        if (ck >= CK) continue;
+        const uint32_t* a = atoms + h2 * 128 + q * 4;
+        reinterpret_cast<uint4*>(scales + ((size_t)bh * CK + ck) * 512)[q] = make_uint4(a[0], a[1], a[2], a[3]);
+    }
+}
+
+// Q/K: grid (ceil(N/128), B*H), 128 * D/64 threads.
+template <int D, bool SMOOTH, bool SEARCH>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ x, int N,
+                                                         const float* __restrict__ kmean,
+                                                         const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
+                                                         uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                         int8_t* __restrict__ ss_off, float* __restrict__ g_out)
+{
+    __shared__ uint4 xs[128 * D / 8];
+    __shared__ uint32_t atoms[2 * 128];
+    __shared__ float rcp[128];
+    fill_rcp_table(rcp);
+    float g, inv_g;
+    tensor_scale(__uint_as_float(*amax_word), g, inv_g);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        g_out[0] = g;
+        g_out[1] = inv_g;
+    }
+    quant_rows_tile<D, SMOOTH, SEARCH>(x, blockIdx.y, blockIdx.x, N, kmean, inv_g, f_lo, f_hi, codes, scales, ss_off,
+                                       xs, atoms, rcp);
+}
+
+// V: grid (ceil(N/128), B*H), 2 D threads.
+template <int D, bool SEARCH>
+__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ x, int N,
                                                       const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                       int8_t* __restrict__ ss_off, float* __restrict__ g_out)
 {
+    __shared__ __align__(16) uint16_t xs[128 * D];
+    __shared__ uint32_t atoms[2 * 128];
+    __shared__ float rcp[128];
+    fill_rcp_table(rcp);
     float g, inv_g;
     tensor_scale(__uint_as_float(*amax_word), g, inv_g);
-    const size_t stride = (size_t)gridDim.x * blockDim.x;
-    const size_t b0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (b0 == 0) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         g_out[0] = g;
         g_out[1] = inv_g;
     }
-    const int NBT = N / 16, D4 = D / 4;
-    const int RT = (D + 127) / 128, CK = (N + 63) / 64, NT = (N + 127) / 128;
-    for (size_t b = b0; b < nblk4; b += stride) {
-        const int c0 = (int)(b % D4) * 4;
-        const size_t rest = b / D4;
-        const int nb = (int)(rest % NBT);
-        const size_t bh = rest / NBT;
-        const uint16_t* p = x + (bh * N + (size_t)nb * 16) * D + c0;
-        uint2 w[16];
+    quant_v_tile<SEARCH>(x, blockIdx.y, blockIdx.x, N, D, inv_g, f_lo, f_hi, codes, scales, ss_off, xs, atoms, rcp);
+}
+
+// ---------------------------------------------------------------------------
+// Fused pre-pass of Q, K and V (one statistics launch, one quantisation launch)
+// ---------------------------------------------------------------------------
+
+// max over this thread's uint4 groups i0, i0 + stride, ... of the bf16
+// magnitude bits (|x| order == unsigned order of bits & 0x7FFF).  Normal
+// (L2-keeping) loads: the quantisation pass reads the same bytes next.
+SA_DEV uint32_t amax_bits_strided(const uint4* __restrict__ x, size_t n16, size_t i0, size_t stride)
+{
+    uint32_t m = 0;
+    size_t i = i0;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 16; i++) w[i] = __ldcs(reinterpret_cast<const uint2*>(p + (size_t)i * D));
+        for (int u = 0; u < 4; u++) v[u] = __ldg(x + i + u * stride);
 #pragma unroll
-        for (int cc = 0; cc < 4; cc++) {
-            float xt[16];
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const uint32_t word = cc < 2 ? w[i].x : w[i].y;
-                xt[i] = __fmul_rn(bf16_bits_to_f32((word >> (16 * (cc & 1))) & 0xFFFFu), inv_g);
-            }
-            uint32_t q0, q1, sc;
-            int off;
-            quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off);
-            const int c = c0 + cc;
-            const size_t crow = bh * D + c;
-            *reinterpret_cast<uint2*>(codes + ((bh * NT + (size_t)(nb >> 3)) * D + c) * 64 + (size_t)(nb & 7) * 8) =
-                make_uint2(q0, q1);
-            const size_t atom = (bh * RT + (size_t)(c >> 7)) * CK + (size_t)(nb >> 2);
-            scales[atom * 512 + sf_atom_offset((uint32_t)(c & 127), (uint32_t)(nb & 3))] = (uint8_t)sc;
-            if (ss_off) ss_off[crow * NBT + nb] = (int8_t)off;
+        for (int u = 0; u < 4; u++) {
+            m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
+            m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
         }
     }
+    for (; i < n16; i += stride) {
+        const uint4 v = __ldg(x + i);
+        m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    }
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+struct PrepassParams {
+    const uint4* q;  // bf16 [B,H,N,D]
+    const uint4* k;
+    const uint4* v;
+    int BH, N, T;
+    int smooth_k;
+    unsigned* amax;    // [3]: Q, K, V (FP32 bits)
+    unsigned* ticket;  // [BH]: K-statistics blocks finished per (b,h)
+    double* psum;
+    float* pmax;
+    float* pmin;
+    float* kmean;
+    int nA;   // amax blocks per tensor
+    int nKS;  // K-statistics blocks (smoothing on)
+    // quantisation
+    uint2* qc;
+    uint8_t* qs;
+    float* qg;
+    uint2* kc;
+    uint8_t* ks;
+    float* kg;
+    uint8_t* vc;
+    uint8_t* vs;
+    float* vg;
+    int f_lo, f_hi;
+};
+
+// With smoothing, blocks [0, nKS) take the K statistics of (b,h, tiles) -- the
+// last block of each (b,h) to finish sums the tile partials in tile order
+// (kmean, K amax).  They come first: they are latency-bound chains, and the
+// amax blocks that follow (nA for Q, then nA for V; without smoothing a third
+// nA for K) stream around them.
+template <int D>
+__global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams p)
+{
+    __shared__ uint32_t red[8];
+    __shared__ int last;
+    __shared__ float fred[8];
+    const int bid = blockIdx.x, tid = threadIdx.x;
+    const size_t n16 = (size_t)p.BH * p.N * D / 8;
+    const bool kstat = p.smooth_k && bid < p.nKS;
+    if (!kstat) {
+        const int a = p.smooth_k ? bid - p.nKS : bid;
+        const int which = a < p.nA ? 0 : (a < 2 * p.nA ? 2 : 1);
+        const uint4* x = which == 0 ? p.q : (which == 2 ? p.v : p.k);
+        const int lb = a - (which == 0 ? 0 : (which == 2 ? p.nA : 2 * p.nA));
+        uint32_t mm = amax_bits_strided(x, n16, (size_t)lb * blockDim.x + tid, (size_t)p.nA * blockDim.x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+        if ((tid & 31) == 0) red[tid >> 5] = mm;
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t b = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); w++) b = max(b, red[w]);
+            if (b >= 0x7F80u) sa_raise(SA_ERR_NONFINITE);
+            atomicMax(&p.amax[which], __float_as_uint(bf16_bits_to_f32(b)));
+        }
+        return;
+    }
+    constexpr int P = D / 2, TPB = 256 / P;
+    const int TB = (p.T + TPB - 1) / TPB;  // blocks per (b,h)
+    const int local = bid;
+    const int bh = local / TB, tb = local % TB;
+    const int cp = tid % P, tile = tb * TPB + tid / P;
+    if (tile < p.T && !kstats_pair<D>(reinterpret_cast<const uint32_t*>(p.k), p.N, p.T, bh, tile, cp, p.psum, p.pmax,
+                                      p.pmin))
+        sa_raise(SA_ERR_NONFINITE);
+    __threadfence();  // partials visible device-wide before the ticket
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(&p.ticket[bh], 1u) == (unsigned)(TB - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    float a = tid < D ? kfinal_channel(p.psum, p.pmax, p.pmin, p.N, p.T, D, bh, tid, p.kmean) : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) fred[tid >> 5] = a;
+    __syncthreads();
+    if (tid == 0) {
+        float b = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); w++) b = fmaxf(b, fred[w]);
+        atomicMax(&p.amax[1], __float_as_uint(b));
+    }
+}
+
+// Tiles [0, BH T): Q; [BH T, 2 BH T): K (smoothed when on); the rest: V.
+// 2 D threads per CTA; the codes and scales are the per-tensor kernels' bytes.
+template <int D, bool SEARCH, bool SMOOTH>
+__global__ void __launch_bounds__(256) prepass_quant_kernel(const PrepassParams p)
+{
+    __shared__ __align__(16) uint16_t xs[128 * D];
+    __shared__ uint32_t atoms[2 * 128];
+    __shared__ float rcp[128];
+    fill_rcp_table(rcp);
+    const int nt = p.BH * p.T;
+    const int bid = blockIdx.x;
+    const int which = bid < nt ? 0 : (bid < 2 * nt ? 1 : 2);
+    const int lb = bid - which * nt;
+    const int bh = lb / p.T, tile = lb % p.T;
+    float g, inv_g;
+    tensor_scale(__uint_as_float(p.amax[which]), g, inv_g);
+    if (lb == 0 && threadIdx.x == 0) {
+        float* go = which == 0 ? p.qg : (which == 1 ? p.kg : p.vg);
+        go[0] = g;
+        go[1] = inv_g;
+    }
+    if (which == 0)
+        quant_rows_tile<D, false, SEARCH>(p.q, bh, tile, p.N, nullptr, inv_g, p.f_lo, p.f_hi, p.qc, p.qs, nullptr,
+                                          reinterpret_cast<uint4*>(xs), atoms, rcp);
+    else if (which == 1)
+        quant_rows_tile<D, SMOOTH, SEARCH>(p.k, bh, tile, p.N, p.kmean, inv_g, p.f_lo, p.f_hi, p.kc, p.ks, nullptr,
+                                           reinterpret_cast<uint4*>(xs), atoms, rcp);
+    else
+        quant_v_tile<SEARCH>(reinterpret_cast<const uint16_t*>(p.v), bh, tile, p.N, D, inv_g, p.f_lo, p.f_hi, p.vc,
+                             p.vs, nullptr, xs, atoms, rcp);
 }
 
 // ---------------------------------------------------------------------------

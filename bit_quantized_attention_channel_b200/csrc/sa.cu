@@ -3,6 +3,7 @@
 // unit so the device status word is a single object.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -160,10 +161,6 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
     const size_t BH = (size_t)B * H;
     const int T = sa_cdiv(N, kTile);
 
-    // padding bytes of the scale atoms must read as zero
-    const bool pad = role == SA_ROLE_V ? (D % 128 != 0 || N % 64 != 0) : (N % 128 != 0);
-    if (pad && cudaMemsetAsync(scales_dev, 0, sa_scales_bytes(B, H, N, D, role), stream) != cudaSuccess)
-        return SA_ERR_CUDA;
     if (cudaMemsetAsync(w.amax, 0, 4, stream) != cudaSuccess) return SA_ERR_CUDA;
 
     float* kmean = k_mean_dev ? k_mean_dev : w.kmean;
@@ -183,23 +180,23 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
     }
 
     const bool ss = mode == SA_SCALE_SEARCH;
+    const dim3 grid((unsigned)T, (unsigned)BH);
     if (role == SA_ROLE_V) {
-        size_t nblk4 = BH * (N / 16) * (D / 4);
-        int grid = grid_for(nblk4, 256);
-        if (ss)
-            quant_v_kernel<true><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk4, N, D, w.amax, f_lo, f_hi,
-                                                           codes_dev, scales_dev, ss_off_dev, g_dev);
-        else
-            quant_v_kernel<false><<<grid, 256, 0, stream>>>((const uint16_t*)x_dev, nblk4, N, D, w.amax, f_lo, f_hi,
-                                                            codes_dev, scales_dev, ss_off_dev, g_dev);
+        const uint16_t* x = (const uint16_t*)x_dev;
+#define SA_QV(DD, SS) quant_v_kernel<DD, SS><<<grid, 2 * DD, 0, stream>>>(x, N, w.amax, f_lo, f_hi, codes_dev, \
+                                                                           scales_dev, ss_off_dev, g_dev)
+        if (D == 128) {
+            if (ss) SA_QV(128, true); else SA_QV(128, false);
+        } else {
+            if (ss) SA_QV(64, true); else SA_QV(64, false);
+        }
+#undef SA_QV
     } else {
-        size_t nblk = BH * N * (D / 16);
-        int grid = grid_for(nblk, 256);
         const uint4* x = (const uint4*)x_dev;
         uint2* c = (uint2*)codes_dev;
 #define SA_QR(DD, SM, SS)                                                                                    \
-    quant_rows_kernel<DD, SM, SS><<<grid, 256, 0, stream>>>(x, nblk, N, T, kmean, w.amax, f_lo, f_hi, c, \
-                                                           scales_dev, ss_off_dev, g_dev)
+    quant_rows_kernel<DD, SM, SS><<<grid, 2 * DD, 0, stream>>>(x, N, kmean, w.amax, f_lo, f_hi, c, scales_dev, \
+                                                              ss_off_dev, g_dev)
         if (D == 128) {
             if (smooth) {
                 if (ss) SA_QR(128, true, true); else SA_QR(128, true, false);
@@ -215,6 +212,122 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
         }
 #undef SA_QR
     }
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+// Workspace of the fused pre-pass: amax words and K tickets (cleared per call),
+// then the K tile partials and channel means.
+struct QkvWs {
+    unsigned* amax;    // [3]
+    unsigned* ticket;  // [B*H]
+    size_t zero_bytes;
+    double* psum;
+    float* pmax;
+    float* pmin;
+    float* kmean;
+    size_t bytes;
+};
+
+static QkvWs qkv_ws_layout(void* base, int B, int H, int N, int D)
+{
+    QkvWs w{};
+    char* p = (char*)base;
+    const size_t BH = (size_t)B * H, T = (size_t)sa_cdiv(N, kTile);
+    w.amax = (unsigned*)p;
+    w.ticket = (unsigned*)(p + 16);
+    w.zero_bytes = sa_align256(16 + BH * sizeof(unsigned));
+    size_t off = w.zero_bytes;
+    w.psum = (double*)(p + off);
+    off += sa_align256(BH * T * D * sizeof(double));
+    w.pmax = (float*)(p + off);
+    off += sa_align256(BH * T * D * sizeof(float));
+    w.pmin = (float*)(p + off);
+    off += sa_align256(BH * T * D * sizeof(float));
+    w.kmean = (float*)(p + off);
+    off += sa_align256(BH * D * sizeof(float));
+    w.bytes = off;
+    return w;
+}
+
+size_t sa_quant_qkv_workspace_size(int B, int H, int N, int D)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    return qkv_ws_layout(nullptr, B, H, N, D).bytes;
+}
+
+sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v_dev, int B, int H, int N, int D,
+                             int smooth_k, sa_scale_mode mode, int f_lo, int f_hi, uint8_t* q_codes_dev,
+                             uint8_t* q_scales_dev, float* q_g_dev, uint8_t* k_codes_dev, uint8_t* k_scales_dev,
+                             float* k_g_dev, float* k_mean_dev, uint8_t* v_codes_dev, uint8_t* v_scales_dev,
+                             float* v_g_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+    if (mode != SA_SCALE_MAX && mode != SA_SCALE_SEARCH) return SA_ERR_INVALID_ARG;
+    if (mode == SA_SCALE_SEARCH && !(f_lo >= -16 && f_lo <= 0 && f_hi > 0 && f_hi <= 16)) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if (N % 16) return SA_ERR_INVALID_ARG;
+    if ((size_t)B * H * N == 0) return SA_OK;
+    if (!q_dev || !k_dev || !v_dev || !q_codes_dev || !q_scales_dev || !q_g_dev || !k_codes_dev || !k_scales_dev ||
+        !k_g_dev || !v_codes_dev || !v_scales_dev || !v_g_dev || !ws_dev)
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || ((uintptr_t)q_codes_dev & 7u) ||
+        ((uintptr_t)k_codes_dev & 7u) || ((uintptr_t)v_codes_dev & 7u) || ((uintptr_t)ws_dev & 255u))
+        return SA_ERR_INVALID_ARG;
+    QkvWs w = qkv_ws_layout(ws_dev, B, H, N, D);
+    if (ws_bytes < w.bytes) return SA_ERR_WORKSPACE;
+    const int BH = B * H, T = sa_cdiv(N, kTile);
+
+    if (cudaMemsetAsync(w.amax, 0, w.zero_bytes, stream) != cudaSuccess) return SA_ERR_CUDA;
+
+    PrepassParams p{};
+    p.q = (const uint4*)q_dev;
+    p.k = (const uint4*)k_dev;
+    p.v = (const uint4*)v_dev;
+    p.BH = BH;
+    p.N = N;
+    p.T = T;
+    p.smooth_k = smooth_k ? 1 : 0;
+    p.amax = w.amax;
+    p.ticket = w.ticket;
+    p.psum = w.psum;
+    p.pmax = w.pmax;
+    p.pmin = w.pmin;
+    p.kmean = k_mean_dev ? k_mean_dev : w.kmean;
+    const size_t n16 = (size_t)BH * N * D / 8;
+    const size_t cap = 148 * 8;
+    p.nA = (int)std::min<size_t>(std::max<size_t>((n16 + 1023) / 1024, 1), cap);
+    const int TPB = 256 / (D / 2);
+    p.nKS = sa_cdiv(T, TPB) * BH;
+    p.qc = (uint2*)q_codes_dev;
+    p.qs = q_scales_dev;
+    p.qg = q_g_dev;
+    p.kc = (uint2*)k_codes_dev;
+    p.ks = k_scales_dev;
+    p.kg = k_g_dev;
+    p.vc = v_codes_dev;
+    p.vs = v_scales_dev;
+    p.vg = v_g_dev;
+    p.f_lo = f_lo;
+    p.f_hi = f_hi;
+
+    const unsigned gs = (unsigned)(2 * p.nA + (p.smooth_k ? p.nKS : p.nA));
+    if (D == 128)
+        prepass_stats_kernel<128><<<gs, 256, 0, stream>>>(p);
+    else
+        prepass_stats_kernel<64><<<gs, 256, 0, stream>>>(p);
+    SA_CHECK_LAUNCH();
+    const unsigned gq = (unsigned)(3 * BH * T);
+    const bool ss = mode == SA_SCALE_SEARCH, sm = p.smooth_k != 0;
+#define SA_PQ(DD, SS, SM) prepass_quant_kernel<DD, SS, SM><<<gq, 2 * DD, 0, stream>>>(p)
+    if (D == 128) {
+        if (ss) { if (sm) SA_PQ(128, true, true); else SA_PQ(128, true, false); }
+        else { if (sm) SA_PQ(128, false, true); else SA_PQ(128, false, false); }
+    } else {
+        if (ss) { if (sm) SA_PQ(64, true, true); else SA_PQ(64, true, false); }
+        else { if (sm) SA_PQ(64, false, true); else SA_PQ(64, false, false); }
+    }
+#undef SA_PQ
     SA_CHECK_LAUNCH();
     return SA_OK;
 }

@@ -123,6 +123,29 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
                          cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * sa_quant_nvfp4_qkv -- the pre-pass of a whole attention call: Q, K and V of
+ * one shape in two kernel launches (one for the statistics of all three
+ * tensors, one for their quantisation) instead of up to three each.
+ * Same operation, arguments and bit-identical outputs as calling
+ * sa_quant_nvfp4 for role Q (smooth 0), K (smooth = smooth_k) and V with the
+ * same mode and offsets; no ScaleSearch offset outputs.
+ *  q_dev, k_dev, v_dev   bf16 [B,H,N,D] inputs.
+ *  *_codes, *_scales, *_g   outputs as sa_quant_nvfp4 for each role.
+ *  k_mean_dev  float [B,H,D] channel means of K (written when smooth_k), may
+ *              be NULL.
+ *  ws_dev      scratch of sa_quant_qkv_workspace_size() bytes (256-byte
+ *              aligned).
+ * Errors: as sa_quant_nvfp4 (argument errors before any launch; non-finite
+ * input in any of the three tensors -> SA_ERR_NONFINITE in the status word).
+ * ------------------------------------------------------------------------ */
+size_t sa_quant_qkv_workspace_size(int B, int H, int N, int D);
+sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v_dev, int B, int H, int N, int D,
+                             int smooth_k, sa_scale_mode mode, int f_lo, int f_hi, uint8_t* q_codes_dev,
+                             uint8_t* q_scales_dev, float* q_g_dev, uint8_t* k_codes_dev, uint8_t* k_scales_dev,
+                             float* k_g_dev, float* k_mean_dev, uint8_t* v_codes_dev, uint8_t* v_scales_dev,
+                             float* v_g_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * sa_quant_nvfp4_noalloc -- sa_quant_nvfp4 without a caller workspace.
  * The pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory: hosts whose device memory is all owned

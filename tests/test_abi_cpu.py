@@ -112,3 +112,16 @@ def test_v_codes_to_logical_roundtrip():
     d, n = 37, 300
     flat = tiled.reshape(-1)
     assert flat[((1 * H + 2) * NT + n // 128) * D * 64 + d * 64 + (n % 128) // 2] == logical[1, 2, d, n // 2]
+
+
+def test_fused_prepass_rejects_bad_arguments(L):
+    n = None
+    ws = L.sa_quant_qkv_workspace_size(1, 2, 256, 128)
+    assert ws >= 256 + 2 * 2 * 128 * (8 + 4 + 4) + 2 * 128 * 4
+    # D unsupported, N not a multiple of 16, bad mode, null pointers: before any launch
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 1, 1, 256, 96, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 2
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 1, 1, 250, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 1
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 1, 1, 256, 128, 1, 7, -2, 6, *([n] * 10), n, 0, n) == 1
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 1, 1, 256, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 1
+    # empty call
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 0, 1, 256, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 0

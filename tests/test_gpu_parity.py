@@ -194,6 +194,28 @@ def test_select_bit_exact_full_size():
     assert np.array_equal(mg.cpu().numpy(), mo)
 
 
+@pytest.mark.parametrize("shape,smooth,mode", [({"N": 4096, "D": 128, "B": 2, "H": 16}, True, "max"),
+                                               ({"N": 416, "D": 64}, True, "search"),
+                                               ({"N": 352, "D": 128}, False, "max"),
+                                               ({"N": 1040, "D": 64, "H": 3}, True, "max")])
+def test_fused_prepass_equals_per_tensor(shape, smooth, mode):
+    """sa_quant_nvfp4_qkv writes the same bytes as three sa_quant_nvfp4 calls."""
+    q, k, v = (t.cuda() for t in inputs("tiny", **shape))
+    ref = (sa.sa_quant_nvfp4(q, "q", mode=mode), sa.sa_quant_nvfp4(k, "k", smooth=smooth, mode=mode),
+           sa.sa_quant_nvfp4(v, "v", mode=mode))
+    got = sa.sa_quant_nvfp4_qkv(q, k, v, smooth=smooth, mode=mode)
+    status_ok()
+    B, H, N, D = q.shape
+    for a, b in zip(got, ref):
+        # V bytes past token N in the last 128-token tile are unspecified
+        assert torch.equal(sa.codes_to_logical(a.codes, B, H, N, D, a.role),
+                           sa.codes_to_logical(b.codes, B, H, N, D, b.role)), a.role
+        assert torch.equal(a.scales, b.scales), a.role
+        assert torch.equal(a.g, b.g), a.role
+    if smooth:
+        assert torch.equal(got[1].k_mean, ref[1].k_mean)
+
+
 # ------------------------------------------------------------------ attention
 ATTN_CASES = [
     ("tiny", {}, False, "max", None),                  # every row compared
