@@ -19,6 +19,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace sa {
 
@@ -277,153 +278,138 @@ __global__ void __launch_bounds__(128) kfinal_kernel(const double* __restrict__ 
 // ---------------------------------------------------------------------------
 
 // ---------------------------------------------------------------------------
-// Tile quantisers: one CTA per (b,h, 128-row tile) of Q/K or (b,h, 128-token
-// tile) of V.  Loads are 16-byte and coalesced; each thread encodes the four
-// blocks of one 64-element chunk, writes their codes as one contiguous 32-byte
-// piece, and assembles the four scale bytes as one word of the tile's scale
-// atoms in shared memory; the atoms (padding zero) go out as 16-byte stores.
-// Per block the arithmetic is quant16, so the bytes equal the per-block
-// kernels'.
+// Tile quantisers: one (b,h, 128-row tile) of Q/K or (b,h, 128-token tile) of
+// V, already in shared memory as row-major bf16 (rows x D, the bytes of one
+// bulk copy: a tile is contiguous in the [B,H,N,D] input).  Each CTA has 2 D
+// threads.  Codes go out coalesced; the four scale bytes of a 64-element
+// chunk form one word of the tile's scale atoms in shared memory, which the
+// caller writes out (padding zero) after a barrier.  Per block the arithmetic
+// is quant16.
 // ---------------------------------------------------------------------------
 
-// Q/K tile: 128 rows x D channels; thread t -> row t / (D/64), chunk t % (D/64).
-// The tile is staged in shared memory by coalesced 16-byte loads (all issued
-// before the first store).  16-byte piece c of row r sits at piece
-// (c & ~7) | ((c ^ (r * CK + c / 8)) & 7) of that row, so that the eight
-// threads of a shared-memory phase (eight different (row, chunk) pairs) read
-// eight different bank groups.
-template <int D, bool SMOOTH, bool SEARCH>
-SA_DEV void quant_rows_tile(const uint4* __restrict__ x, size_t bh, int tile, int N, const float* __restrict__ kmean,
-                            float inv_g, int f_lo, int f_hi, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
-                            int8_t* __restrict__ ss_off, uint4* xs /* shared, 128 * D / 8 */,
-                            uint32_t* atoms /* shared, CK * 128 words */, const float* rcp /* shared, filled */)
+// Bytes of tile `tile` of a [*, N, D] bf16 tensor slice bh, and its address.
+SA_DEV uint32_t tile_bytes(int N, int D, int tile) { return (uint32_t)(min(kTile, N - tile * kTile) * D * 2); }
+SA_DEV const void* tile_src(const void* x, size_t bh, int N, int D, int tile)
 {
-    constexpr int CK = D / 64, NB = D / 16, RP = D / 8;  // 16-byte pieces per row
-    constexpr int NTH = 128 * CK, PER = 128 * RP / NTH;  // threads, pieces per thread
+    return (const uint8_t*)x + ((bh * N + (size_t)tile * kTile) * D) * 2;
+}
+
+// Q/K: thread t encodes blocks b = t + 2 D k (k = 0..3), row b / (D/16),
+// block j = b % (D/16).  The eight threads of a shared-memory phase read
+// eight consecutive blocks (32 bytes each); thread t reads the half
+// ((t >> 2) & 1) first, so each phase touches eight different bank groups.
+template <int D, bool SMOOTH, bool SEARCH>
+SA_DEV void quant_rows_smem(const uint4* xs, size_t bh, int tile, int N, const float* __restrict__ kmean, float inv_g,
+                            int f_lo, int f_hi, uint2* __restrict__ codes, int8_t* __restrict__ ss_off,
+                            uint32_t* atoms /* shared, D/64 * 128 words */, const float* rcp)
+{
+    constexpr int NB = D / 16, RP = D / 8, NTH = 2 * D;
     const int t = threadIdx.x;
-    const int r = t / CK, ck = t % CK;
-    const int n = tile * 128 + r;
-    const int T = (N + 127) / 128;
-    const int rows = min(128, N - tile * 128);
-    {
-        const uint4* src = x + (bh * N + (size_t)tile * 128) * RP;
-        uint4 u[PER];
+    const int rows = min(kTile, N - tile * kTile);
+    const int sw = (t >> 2) & 1;
+    float km[16];  // NTH is a multiple of NB: the block column j is t % NB on every pass
+    if (SMOOTH) {
 #pragma unroll
-        for (int k = 0; k < PER; k++) {
-            const int i = t + k * NTH;
-            u[k] = i < rows * RP ? __ldcs(src + i) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int k = 0; k < PER; k++) {
-            const int i = t + k * NTH, rr = i / RP, c = i % RP;
-            xs[rr * RP + ((c & ~7) | ((c ^ (rr * CK + c / 8)) & 7))] = u[k];
-        }
+        for (int i = 0; i < 16; i++) km[i] = __ldg(kmean + bh * D + (t % NB) * 16 + i);
     }
-    for (int i = t; i < CK * 128; i += blockDim.x) atoms[i] = 0u;
-    __syncthreads();
-    if (n < N) {
-        const size_t row = bh * N + n;
-        uint32_t word = 0;
-        uint2 cw[4];
-        uint32_t offw = 0;
-#pragma unroll
-        for (int jb = 0; jb < 4; jb++) {
-            uint4 ua, ub;
-            {
-                const int c0 = ck * 8 + 2 * jb, c1 = c0 + 1;
-                ua = xs[r * RP + ((c0 & ~7) | ((c0 ^ (r * CK + ck)) & 7))];
-                ub = xs[r * RP + ((c1 & ~7) | ((c1 ^ (r * CK + ck)) & 7))];
-            }
-            const uint32_t w[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-            const int j = ck * 4 + jb;
+#pragma unroll 1
+    for (int k = 0; k < 4; k++) {
+        const int b = t + k * NTH, r = b / NB, j = b % NB;
+        uint32_t sc = 0;
+        if (r < rows) {
+            const uint4 pa = xs[r * RP + 2 * j + sw], pb = xs[r * RP + 2 * j + 1 - sw];
+            const uint4 lo = sw ? pb : pa, hi = sw ? pa : pb;
+            const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
             float xt[16];
 #pragma unroll
             for (int i = 0; i < 16; i += 2) {
                 float v0 = __uint_as_float(w[i >> 1] << 16), v1 = __uint_as_float(w[i >> 1] & 0xFFFF0000u);
                 if (SMOOTH) {
-                    v0 = __fsub_rn(v0, __ldg(kmean + bh * D + j * 16 + i));
-                    v1 = __fsub_rn(v1, __ldg(kmean + bh * D + j * 16 + i + 1));
+                    v0 = __fsub_rn(v0, km[i]);
+                    v1 = __fsub_rn(v1, km[i + 1]);
                 }
                 mul2_rn(v0, v1, inv_g, xt[i], xt[i + 1]);
             }
-            uint32_t c0, c1, sc;
+            uint32_t c0, c1;
             int off;
             quant16<SEARCH>(xt, f_lo, f_hi, c0, c1, sc, off, rcp);
-            cw[jb] = make_uint2(c0, c1);
-            word |= sc << (8 * jb);
-            offw |= ((uint32_t)(uint8_t)(int8_t)off) << (8 * jb);
+            const size_t row = bh * N + (size_t)tile * kTile + r;
+            codes[row * NB + j] = make_uint2(c0, c1);
+            if (ss_off) ss_off[row * NB + j] = (int8_t)off;
         }
-        uint4* dst = reinterpret_cast<uint4*>(codes + row * NB + ck * 4);
-        dst[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
-        dst[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
-        atoms[ck * 128 + (r & 31) * 4 + (r >> 5)] = word;
-        if (ss_off) *reinterpret_cast<uint32_t*>(ss_off + row * NB + ck * 4) = offw;
-    }
-    __syncthreads();
-    // atom (bh, tile, ck): 512 bytes = 32 x uint4
-    for (int i = t; i < CK * 32; i += blockDim.x) {
-        const int ck2 = i / 32, q = i % 32;
-        const uint32_t* a = atoms + ck2 * 128 + q * 4;
-        reinterpret_cast<uint4*>(scales + (((size_t)bh * T + tile) * CK + ck2) * 512)[q] = make_uint4(a[0], a[1], a[2], a[3]);
+        // the four lanes t & ~3 .. t | 3 hold blocks 4 m .. 4 m + 3 of row r
+        uint32_t word = sc << (8 * (j & 3));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        if ((j & 3) == 0) atoms[(j >> 2) * 128 + (r & 31) * 4 + (r >> 5)] = word;
     }
 }
 
-// V tile: tokens 128 tile .. +127 x D channels, staged in shared memory
-// (row-major bf16, 128 x D); thread t -> channel t % D, token half t / D
-// (blocks 4 half .. 4 half + 3 of the tile).
-template <bool SEARCH>
-SA_DEV void quant_v_tile(const uint16_t* __restrict__ x, size_t bh, int tile, int N, int D, float inv_g, int f_lo,
-                         int f_hi, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                         int8_t* __restrict__ ss_off, uint16_t* xs /* shared, 128 * D */,
-                         uint32_t* atoms /* shared, 2 * 128 words */, const float* rcp /* shared, filled */)
+// Q/K scale atoms (bh, tile, chunk): 512 bytes = 32 x uint4 each.
+template <int D>
+SA_DEV void store_rows_atoms(const uint32_t* atoms, size_t bh, int tile, int T, uint8_t* __restrict__ scales)
+{
+    constexpr int CK = D / 64;
+    for (int i = threadIdx.x; i < CK * 32; i += blockDim.x) {
+        const int ck = i / 32, q = i % 32;
+        const uint32_t* a = atoms + ck * 128 + q * 4;
+        reinterpret_cast<uint4*>(scales + (((size_t)bh * T + tile) * CK + ck) * 512)[q] = make_uint4(a[0], a[1], a[2], a[3]);
+    }
+}
+
+// V: thread t -> channel t % D, token half t / D (blocks 4 half .. 4 half + 3
+// of the tile, 16 tokens each).  Atom words of padded rows are written zero.
+template <int D, bool SEARCH>
+SA_DEV void quant_v_smem(const uint16_t* xs, size_t bh, int tile, int N, float inv_g, int f_lo, int f_hi,
+                         uint8_t* __restrict__ codes, int8_t* __restrict__ ss_off,
+                         uint32_t* atoms /* shared, 2 * 128 words */, const float* rcp)
 {
     const int t = threadIdx.x;
-    const int NT = (N + 127) / 128, CK = (N + 63) / 64, NBT = N / 16;
-    const int rows = min(128, N - tile * 128);
-    // coalesced 16-byte loads of the tile
-    const uint4* src = reinterpret_cast<const uint4*>(x + (bh * N + (size_t)tile * 128) * D);
-    for (int i = t; i < rows * D / 8; i += blockDim.x) reinterpret_cast<uint4*>(xs)[i] = __ldcs(src + i);
-    for (int i = t; i < 256; i += blockDim.x) atoms[i] = 0u;
-    __syncthreads();
+    const int NT = (N + 127) / 128, NBT = N / 16;
+    const int rows = min(kTile, N - tile * kTile);
     const int c = t % D, half = t / D;
-    if (half < 2) {
-        uint32_t word = 0, offw = 0;
-        uint2 cw[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
+    uint32_t word = 0, offw = 0;
+    uint2 cw[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
 #pragma unroll
-        for (int jb = 0; jb < 4; jb++) {
-            const int tok0 = half * 64 + jb * 16;
-            if (tok0 >= rows) break;
-            float xt[16];
+    for (int jb = 0; jb < 4; jb++) {
+        const int tok0 = half * 64 + jb * 16;
+        if (tok0 >= rows) break;
+        float xt[16];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2)
-                mul2_rn(bf16_bits_to_f32(xs[(tok0 + i) * D + c]), bf16_bits_to_f32(xs[(tok0 + i + 1) * D + c]), inv_g,
-                        xt[i], xt[i + 1]);
-            uint32_t q0, q1, sc;
-            int off;
-            quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off, rcp);
-            cw[jb] = make_uint2(q0, q1);
-            word |= sc << (8 * jb);
-            offw |= ((uint32_t)(uint8_t)(int8_t)off) << (8 * jb);
+        for (int i = 0; i < 16; i += 2)
+            mul2_rn(bf16_bits_to_f32(xs[(tok0 + i) * D + c]), bf16_bits_to_f32(xs[(tok0 + i + 1) * D + c]), inv_g,
+                    xt[i], xt[i + 1]);
+        uint32_t q0, q1, sc;
+        int off;
+        quant16<SEARCH>(xt, f_lo, f_hi, q0, q1, sc, off, rcp);
+        cw[jb] = make_uint2(q0, q1);
+        word |= sc << (8 * jb);
+        offw |= ((uint32_t)(uint8_t)(int8_t)off) << (8 * jb);
+    }
+    const int nblk_here = min(4, max(0, (rows - half * 64) / 16));
+    if (nblk_here > 0) {
+        uint8_t* dst = codes + (((size_t)bh * NT + tile) * D + c) * 64 + half * 32;
+        if (nblk_here == 4) {
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
+        } else {
+            for (int jb = 0; jb < nblk_here; jb++) reinterpret_cast<uint2*>(dst)[jb] = cw[jb];
         }
-        const int nblk_here = min(4, max(0, (rows - half * 64) / 16));
-        if (nblk_here > 0) {
-            uint8_t* dst = codes + (((size_t)bh * NT + tile) * D + c) * 64 + half * 32;
-            if (nblk_here == 4) {
-                reinterpret_cast<uint4*>(dst)[0] = make_uint4(cw[0].x, cw[0].y, cw[1].x, cw[1].y);
-                reinterpret_cast<uint4*>(dst)[1] = make_uint4(cw[2].x, cw[2].y, cw[3].x, cw[3].y);
-            } else {
-                for (int jb = 0; jb < nblk_here; jb++) reinterpret_cast<uint2*>(dst)[jb] = cw[jb];
-            }
-            atoms[half * 128 + (c & 31) * 4 + ((c & 127) >> 5)] = word;
-            if (ss_off) {
-                int8_t* so = ss_off + ((size_t)bh * D + c) * NBT + tile * 8 + half * 4;
-                for (int jb = 0; jb < nblk_here; jb++) so[jb] = (int8_t)(offw >> (8 * jb));
-            }
+        if (ss_off) {
+            int8_t* so = ss_off + ((size_t)bh * D + c) * NBT + tile * 8 + half * 4;
+            for (int jb = 0; jb < nblk_here; jb++) so[jb] = (int8_t)(offw >> (8 * jb));
         }
     }
-    __syncthreads();
-    // atoms (bh, channel tile 0, chunks 2 tile, 2 tile + 1), only chunks inside N
-    for (int i = t; i < 64; i += blockDim.x) {
+    // channel rows D..127 of the atom stay zero (written by the caller once)
+    atoms[half * 128 + (c & 31) * 4 + ((c & 127) >> 5)] = word;
+}
+
+// V scale atoms (bh, channel tile 0, chunks 2 tile, 2 tile + 1), only chunks
+// inside N.
+SA_DEV void store_v_atoms(const uint32_t* atoms, size_t bh, int tile, int N, uint8_t* __restrict__ scales)
+{
+    const int CK = (N + 63) / 64;
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) {
         const int h2 = i / 32, q = i % 32;
         const int ck = 2 * tile + h2;
         if (ck >= CK) continue;
@@ -432,15 +418,36 @@ SA_DEV void quant_v_tile(const uint16_t* __restrict__ x, size_t bh, int tile, in
     }
 }
 
-// Q/K: grid (ceil(N/128), B*H), 128 * D/64 threads.
-template <int D, bool SMOOTH, bool SEARCH>
-__global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict__ x, int N,
-                                                         const float* __restrict__ kmean,
-                                                         const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
-                                                         uint2* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                         int8_t* __restrict__ ss_off, float* __restrict__ g_out)
+// One CTA = one tile: a single bulk copy into shared memory, then the tile
+// quantiser.  Returns false (status raised) when the copy never lands.
+SA_DEV bool load_tile_once(void* xs, const void* src, uint32_t bytes, uint64_t* bar)
 {
-    __shared__ uint4 xs[128 * D / 8];
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(bar, bytes);
+        bulk_load(xs, src, bytes, bar);
+    }
+    if (__syncthreads_or(!mbar_wait(bar, 0))) {
+        if (threadIdx.x == 0) sa_raise(SA_ERR_TIMEOUT);
+        return false;
+    }
+    return true;
+}
+
+// Q/K: grid (ceil(N/128), B*H), 2 D threads.
+template <int D, bool SMOOTH, bool SEARCH>
+__global__ void __launch_bounds__(2 * D) quant_rows_kernel(const uint4* __restrict__ x, int N,
+                                                           const float* __restrict__ kmean,
+                                                           const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
+                                                           uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                           int8_t* __restrict__ ss_off, float* __restrict__ g_out)
+{
+    __shared__ __align__(128) uint4 xs[kTile * D / 8];
+    __shared__ __align__(8) uint64_t bar;
     __shared__ uint32_t atoms[2 * 128];
     __shared__ float rcp[128];
     fill_rcp_table(rcp);
@@ -450,59 +457,63 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint4* __restrict
         g_out[0] = g;
         g_out[1] = inv_g;
     }
-    quant_rows_tile<D, SMOOTH, SEARCH>(x, blockIdx.y, blockIdx.x, N, kmean, inv_g, f_lo, f_hi, codes, scales, ss_off,
-                                       xs, atoms, rcp);
+    const int tile = blockIdx.x;
+    if (!load_tile_once(xs, tile_src(x, blockIdx.y, N, D, tile), tile_bytes(N, D, tile), &bar)) return;
+    quant_rows_smem<D, SMOOTH, SEARCH>(xs, blockIdx.y, tile, N, kmean, inv_g, f_lo, f_hi, codes, ss_off, atoms, rcp);
+    __syncthreads();
+    store_rows_atoms<D>(atoms, blockIdx.y, tile, (N + kTile - 1) / kTile, scales);
 }
 
 // V: grid (ceil(N/128), B*H), 2 D threads.
 template <int D, bool SEARCH>
-__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ x, int N,
-                                                      const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
-                                                      uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                      int8_t* __restrict__ ss_off, float* __restrict__ g_out)
+__global__ void __launch_bounds__(2 * D) quant_v_kernel(const uint16_t* __restrict__ x, int N,
+                                                        const unsigned* __restrict__ amax_word, int f_lo, int f_hi,
+                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                        int8_t* __restrict__ ss_off, float* __restrict__ g_out)
 {
-    __shared__ __align__(16) uint16_t xs[128 * D];
+    __shared__ __align__(128) uint16_t xs[kTile * D];
+    __shared__ __align__(8) uint64_t bar;
     __shared__ uint32_t atoms[2 * 128];
     __shared__ float rcp[128];
     fill_rcp_table(rcp);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) atoms[i] = 0u;
     float g, inv_g;
     tensor_scale(__uint_as_float(*amax_word), g, inv_g);
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         g_out[0] = g;
         g_out[1] = inv_g;
     }
-    quant_v_tile<SEARCH>(x, blockIdx.y, blockIdx.x, N, D, inv_g, f_lo, f_hi, codes, scales, ss_off, xs, atoms, rcp);
+    const int tile = blockIdx.x;
+    if (!load_tile_once(xs, tile_src(x, blockIdx.y, N, D, tile), tile_bytes(N, D, tile), &bar)) return;
+    quant_v_smem<D, SEARCH>(xs, blockIdx.y, tile, N, inv_g, f_lo, f_hi, codes, ss_off, atoms, rcp);
+    __syncthreads();
+    store_v_atoms(atoms, blockIdx.y, tile, N, scales);
 }
 
 // ---------------------------------------------------------------------------
 // Fused pre-pass of Q, K and V (one statistics launch, one quantisation launch)
 // ---------------------------------------------------------------------------
 
-// max over this thread's uint4 groups i0, i0 + stride, ... of the bf16
-// magnitude bits (|x| order == unsigned order of bits & 0x7FFF).  Normal
-// (L2-keeping) loads: the quantisation pass reads the same bytes next.
-SA_DEV uint32_t amax_bits_strided(const uint4* __restrict__ x, size_t n16, size_t i0, size_t stride)
+// max over the uint4 groups i0 + u stride (u < kAmaxPer) of the bf16
+// magnitude bits (|x| order == unsigned order of bits & 0x7FFF); all loads
+// are issued before the first use.  Normal (L2-keeping) loads: the
+// quantisation pass reads the same bytes next.
+constexpr int kAmaxPer = 8;
+SA_DEV uint32_t amax_bits_batch(const uint4* __restrict__ x, size_t n16, size_t i0, size_t stride)
 {
-    uint32_t m = 0;
-    size_t i = i0;
-    for (; i + 3 * stride < n16; i += 4 * stride) {
-        uint4 v[4];
+    uint4 v[kAmaxPer];
 #pragma unroll
-        for (int u = 0; u < 4; u++) v[u] = __ldg(x + i + u * stride);
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
-            m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
-            m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
-            m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
-        }
+    for (int u = 0; u < kAmaxPer; u++) {
+        const size_t i = i0 + u * stride;
+        v[u] = i < n16 ? __ldg(x + i) : make_uint4(0, 0, 0, 0);
     }
-    for (; i < n16; i += stride) {
-        const uint4 v = __ldg(x + i);
-        m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
-        m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
-        m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
-        m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kAmaxPer; u++) {
+        m = __vmaxu2(m, v[u].x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v[u].y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v[u].z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, v[u].w & 0x7FFF7FFFu);
     }
     return max(m & 0xFFFFu, m >> 16);
 }
@@ -519,8 +530,8 @@ struct PrepassParams {
     float* pmax;
     float* pmin;
     float* kmean;
-    int nA;   // amax blocks per tensor
-    int nKS;  // K-statistics blocks (smoothing on)
+    int nA;   // amax blocks per tensor (nA * 256 * kAmaxPer >= B H N D / 8)
+    int nKS;  // K-statistics blocks (smoothing on): B H T, one tile each
     // quantisation
     uint2* qc;
     uint8_t* qs;
@@ -534,17 +545,46 @@ struct PrepassParams {
     int f_lo, f_hi;
 };
 
-// With smoothing, blocks [0, nKS) take the K statistics of (b,h, tiles) -- the
-// last block of each (b,h) to finish sums the tile partials in tile order
-// (kmean, K amax).  They come first: they are latency-bound chains, and the
-// amax blocks that follow (nA for Q, then nA for V; without smoothing a third
-// nA for K) stream around them.
+// Channel c of one K tile in shared memory (rows x D bf16, rows % 16 == 0):
+// FP64 sum over the tokens in ascending order, FP32 max and min.  A
+// non-finite input makes the FP64 sum non-finite (the sum of at most 2^20
+// finite bf16 values cannot overflow FP64), which the caller checks.
+template <int D>
+SA_DEV void kstats_channel_smem(const uint16_t* xs, int rows, int c, double& s, float& mx, float& mn)
+{
+    s = 0.0;
+    mx = -INFINITY;
+    mn = INFINITY;
+    for (int r0 = 0; r0 < rows; r0 += 16) {
+        float x[16];
+#pragma unroll
+        for (int u = 0; u < 16; u++) x[u] = bf16_bits_to_f32(xs[(r0 + u) * D + c]);
+#pragma unroll
+        for (int u = 0; u < 16; u++) {
+            s = __dadd_rn(s, (double)x[u]);  // tokens in ascending order
+            mx = fmaxf(mx, x[u]);
+            mn = fminf(mn, x[u]);
+        }
+    }
+}
+
+// With smoothing, blocks [0, B H T) take the K statistics of one (b,h, tile)
+// each: one bulk copy of the tile into shared memory, then one FP64 chain per
+// channel.  The last block of each (b,h) to finish (a ticket) reduces the
+// tile partials: threads [0, D) sum them in tile order (mean), threads
+// [D, 2 D) take their max and min (order-free), and the K amax is
+// max(fl(max - mean), fl(mean - min)) over the channels.  The K blocks come
+// first; the amax blocks that follow (nA for Q, then nA for V; without
+// smoothing a third nA for K) stream around them.
 template <int D>
 __global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams p)
 {
+    extern __shared__ __align__(128) uint16_t ks_tile[];  // kTile x D bf16 (K blocks only)
+    __shared__ __align__(8) uint64_t bar;
     __shared__ uint32_t red[8];
     __shared__ int last;
     __shared__ float fred[8];
+    __shared__ float mu_s[128], mx_s[128], mn_s[128];
     const int bid = blockIdx.x, tid = threadIdx.x;
     const size_t n16 = (size_t)p.BH * p.N * D / 8;
     const bool kstat = p.smooth_k && bid < p.nKS;
@@ -553,7 +593,8 @@ __global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams 
         const int which = a < p.nA ? 0 : (a < 2 * p.nA ? 2 : 1);
         const uint4* x = which == 0 ? p.q : (which == 2 ? p.v : p.k);
         const int lb = a - (which == 0 ? 0 : (which == 2 ? p.nA : 2 * p.nA));
-        uint32_t mm = amax_bits_strided(x, n16, (size_t)lb * blockDim.x + tid, (size_t)p.nA * blockDim.x);
+        // nA * 256 * kAmaxPer >= n16: one batch covers the tensor
+        uint32_t mm = amax_bits_batch(x, n16, (size_t)lb * blockDim.x + tid, (size_t)p.nA * blockDim.x);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, o));
         if ((tid & 31) == 0) red[tid >> 5] = mm;
@@ -566,21 +607,62 @@ __global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams 
         }
         return;
     }
-    constexpr int P = D / 2, TPB = 256 / P;
-    const int TB = (p.T + TPB - 1) / TPB;  // blocks per (b,h)
-    const int local = bid;
-    const int bh = local / TB, tb = local % TB;
-    const int cp = tid % P, tile = tb * TPB + tid / P;
-    if (tile < p.T && !kstats_pair<D>(reinterpret_cast<const uint32_t*>(p.k), p.N, p.T, bh, tile, cp, p.psum, p.pmax,
-                                      p.pmin))
-        sa_raise(SA_ERR_NONFINITE);
+    const int bh = bid / p.T, tile = bid - bh * p.T;
+    const int rows = min(kTile, p.N - tile * kTile);
+    if (!load_tile_once(ks_tile, tile_src(p.k, bh, p.N, D, tile), tile_bytes(p.N, D, tile), &bar)) return;
+    if (tid < D) {
+        double sum;
+        float mx, mn;
+        kstats_channel_smem<D>(ks_tile, rows, tid, sum, mx, mn);
+        if (!isfinite(sum)) sa_raise(SA_ERR_NONFINITE);
+        const size_t o = ((size_t)bh * p.T + tile) * D + tid;
+        p.psum[o] = sum;
+        p.pmax[o] = mx;
+        p.pmin[o] = mn;
+    }
     __threadfence();  // partials visible device-wide before the ticket
     __syncthreads();
-    if (tid == 0) last = atomicAdd(&p.ticket[bh], 1u) == (unsigned)(TB - 1);
+    if (tid == 0) last = atomicAdd(&p.ticket[bh], 1u) == (unsigned)(p.T - 1);
     __syncthreads();
     if (!last) return;
     __threadfence();
-    float a = tid < D ? kfinal_channel(p.psum, p.pmax, p.pmin, p.N, p.T, D, bh, tid, p.kmean) : 0.0f;
+    const int T = p.T;
+    if (tid < D) {
+        double total = 0.0;
+        for (int t0 = 0; t0 < T; t0 += 16) {
+            double ps[16];
+#pragma unroll
+            for (int u = 0; u < 16; u++) ps[u] = __ldcg(p.psum + ((size_t)bh * T + min(t0 + u, T - 1)) * D + tid);
+#pragma unroll
+            for (int u = 0; u < 16; u++)
+                if (t0 + u < T) total = __dadd_rn(total, ps[u]);  // tiles in ascending order
+        }
+        const float mu = __double2float_rn(__ddiv_rn(total, (double)p.N));
+        p.kmean[(size_t)bh * D + tid] = mu;
+        mu_s[tid] = mu;
+    } else if (tid < 2 * D) {
+        const int c = tid - D;
+        float mx = -INFINITY, mn = INFINITY;
+        for (int t0 = 0; t0 < T; t0 += 16) {
+            float px[16], pn[16];
+#pragma unroll
+            for (int u = 0; u < 16; u++) {
+                const size_t o = ((size_t)bh * T + min(t0 + u, T - 1)) * D + c;
+                px[u] = __ldcg(p.pmax + o);
+                pn[u] = __ldcg(p.pmin + o);
+            }
+#pragma unroll
+            for (int u = 0; u < 16; u++) {
+                mx = fmaxf(mx, px[u]);  // clamped repeats of tile T - 1 change nothing
+                mn = fminf(mn, pn[u]);
+            }
+        }
+        mx_s[c] = mx;
+        mn_s[c] = mn;
+    }
+    __syncthreads();
+    float a = 0.0f;
+    if (tid < D) a = fmaxf(fmaxf(__fsub_rn(mx_s[tid], mu_s[tid]), __fsub_rn(mu_s[tid], mn_s[tid])), 0.0f);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     if ((tid & 31) == 0) fred[tid >> 5] = a;
@@ -592,36 +674,92 @@ __global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams 
     }
 }
 
-// Tiles [0, BH T): Q; [BH T, 2 BH T): K (smoothed when on); the rest: V.
-// 2 D threads per CTA; the codes and scales are the per-tensor kernels' bytes.
+// Persistent quantisation of Q, K and V: gridDim.x CTAs of 2 D threads walk
+// the 3 B H T tiles with stride gridDim.x, in the order V, Q, K (the
+// statistics pass streams K first, so V and Q are the likelier L2 hits).
+// Each CTA double-buffers its tiles in shared memory: the bulk copy of the
+// next tile is in flight while the current one is encoded.
+template <int D>
+struct PqSmem {
+    uint4 x[2][kTile * D / 8];
+    uint64_t full[2];
+    uint32_t atoms[2 * 128];
+    float rcp[128];
+};
+
 template <int D, bool SEARCH, bool SMOOTH>
-__global__ void __launch_bounds__(256) prepass_quant_kernel(const PrepassParams p)
+__global__ void __launch_bounds__(2 * D) prepass_quant_kernel(const PrepassParams p)
 {
-    __shared__ __align__(16) uint16_t xs[128 * D];
-    __shared__ uint32_t atoms[2 * 128];
-    __shared__ float rcp[128];
-    fill_rcp_table(rcp);
-    const int nt = p.BH * p.T;
-    const int bid = blockIdx.x;
-    const int which = bid < nt ? 0 : (bid < 2 * nt ? 1 : 2);
-    const int lb = bid - which * nt;
-    const int bh = lb / p.T, tile = lb % p.T;
-    float g, inv_g;
-    tensor_scale(__uint_as_float(p.amax[which]), g, inv_g);
-    if (lb == 0 && threadIdx.x == 0) {
-        float* go = which == 0 ? p.qg : (which == 1 ? p.kg : p.vg);
-        go[0] = g;
-        go[1] = inv_g;
+    extern __shared__ __align__(128) uint8_t pq_raw[];
+    PqSmem<D>& s = *reinterpret_cast<PqSmem<D>*>(pq_raw);
+    const int nt = p.BH * p.T, total = 3 * nt;
+    // tile j -> tensor (0 Q, 1 K, 2 V), bh, tile
+    auto decode = [&](int j, int& which, int& bh, int& tile) {
+        const int w = j / nt, lb = j - w * nt;
+        which = w == 0 ? 2 : w - 1;
+        bh = lb / p.T;
+        tile = lb - bh * p.T;
+    };
+    auto issue = [&](int j, int b) {
+        int which, bh, tile;
+        decode(j, which, bh, tile);
+        const void* x = which == 0 ? (const void*)p.q : (which == 1 ? (const void*)p.k : (const void*)p.v);
+        const uint32_t bytes = tile_bytes(p.N, D, tile);
+        mbar_expect_tx(&s.full[b], bytes);
+        bulk_load(s.x[b], tile_src(x, bh, p.N, D, tile), bytes, &s.full[b]);
+    };
+    fill_rcp_table(s.rcp);
+    if (threadIdx.x == 0) {
+        mbar_init(&s.full[0], 1);
+        mbar_init(&s.full[1], 1);
+        fence_mbar_init();
     }
-    if (which == 0)
-        quant_rows_tile<D, false, SEARCH>(p.q, bh, tile, p.N, nullptr, inv_g, p.f_lo, p.f_hi, p.qc, p.qs, nullptr,
-                                          reinterpret_cast<uint4*>(xs), atoms, rcp);
-    else if (which == 1)
-        quant_rows_tile<D, SMOOTH, SEARCH>(p.k, bh, tile, p.N, p.kmean, inv_g, p.f_lo, p.f_hi, p.kc, p.ks, nullptr,
-                                           reinterpret_cast<uint4*>(xs), atoms, rcp);
-    else
-        quant_v_tile<SEARCH>(reinterpret_cast<const uint16_t*>(p.v), bh, tile, p.N, D, inv_g, p.f_lo, p.f_hi, p.vc,
-                             p.vs, nullptr, xs, atoms, rcp);
+    __syncthreads();
+    int j = blockIdx.x;
+    if (threadIdx.x == 0 && j < total) issue(j, 0);
+    float g[3], inv_g[3];
+#pragma unroll
+    for (int w = 0; w < 3; w++) tensor_scale(__uint_as_float(p.amax[w]), g[w], inv_g[w]);
+    if (blockIdx.x == 0 && threadIdx.x < 3) {
+        float* go = threadIdx.x == 0 ? p.qg : (threadIdx.x == 1 ? p.kg : p.vg);
+        go[0] = g[threadIdx.x];
+        go[1] = inv_g[threadIdx.x];
+    }
+    for (int it = 0; j < total; it++, j += gridDim.x) {
+        const int b = it & 1;
+        const bool next = j + (int)gridDim.x < total;
+        // buffer b ^ 1 was released by the barrier that ended the previous tile
+        if (threadIdx.x == 0 && next) issue(j + gridDim.x, b ^ 1);
+        if (__syncthreads_or(!mbar_wait(&s.full[b], (it >> 1) & 1))) {
+            if (threadIdx.x == 0) {
+                sa_raise(SA_ERR_TIMEOUT);
+                if (next) mbar_wait(&s.full[b ^ 1], ((it + 1) >> 1) & 1);  // bounded: the copy in flight
+            }
+            return;
+        }
+        int which, bh, tile;
+        decode(j, which, bh, tile);
+        if (which == 2) {
+            for (int i = D + threadIdx.x; i < 128; i += blockDim.x) {  // channel rows D..127 of the atoms
+                s.atoms[(i & 31) * 4 + (i >> 5)] = 0u;
+                s.atoms[128 + (i & 31) * 4 + (i >> 5)] = 0u;
+            }
+            quant_v_smem<D, SEARCH>(reinterpret_cast<const uint16_t*>(s.x[b]), bh, tile, p.N, inv_g[2], p.f_lo,
+                                    p.f_hi, p.vc, nullptr, s.atoms, s.rcp);
+            __syncthreads();
+            store_v_atoms(s.atoms, bh, tile, p.N, p.vs);
+        } else if (which == 0) {
+            quant_rows_smem<D, false, SEARCH>(s.x[b], bh, tile, p.N, nullptr, inv_g[0], p.f_lo, p.f_hi, p.qc, nullptr,
+                                              s.atoms, s.rcp);
+            __syncthreads();
+            store_rows_atoms<D>(s.atoms, bh, tile, p.T, p.qs);
+        } else {
+            quant_rows_smem<D, SMOOTH, SEARCH>(s.x[b], bh, tile, p.N, p.kmean, inv_g[1], p.f_lo, p.f_hi, p.kc,
+                                               nullptr, s.atoms, s.rcp);
+            __syncthreads();
+            store_rows_atoms<D>(s.atoms, bh, tile, p.T, p.ks);
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -31,7 +31,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 3-D byte tensor {d0 (contiguous), d1, d2}; box {b0, b1, 1}.
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count()
 {
@@ -45,6 +44,7 @@ int sm_count()
     return n;
 }
 
+// 3-D byte tensor {d0 (contiguous), d1, d2}; box {b0, b1, 1}.
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                  uint32_t b1, CUtensorMapSwizzle swz)
 {
@@ -295,10 +295,9 @@ sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v
     p.pmin = w.pmin;
     p.kmean = k_mean_dev ? k_mean_dev : w.kmean;
     const size_t n16 = (size_t)BH * N * D / 8;
-    const size_t cap = 148 * 8;
-    p.nA = (int)std::min<size_t>(std::max<size_t>((n16 + 1023) / 1024, 1), cap);
-    const int TPB = 256 / (D / 2);
-    p.nKS = sa_cdiv(T, TPB) * BH;
+    // one batch of kAmaxPer 16-byte loads per amax thread
+    p.nA = (int)std::max<size_t>((n16 + 256 * kAmaxPer - 1) / (256 * kAmaxPer), 1);
+    p.nKS = BH * T;
     p.qc = (uint2*)q_codes_dev;
     p.qs = q_scales_dev;
     p.qg = q_g_dev;
@@ -312,14 +311,28 @@ sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v
     p.f_hi = f_hi;
 
     const unsigned gs = (unsigned)(2 * p.nA + (p.smooth_k ? p.nKS : p.nA));
+    const size_t ks_smem = (size_t)kTile * D * 2;  // one K tile (smoothing blocks)
     if (D == 128)
-        prepass_stats_kernel<128><<<gs, 256, 0, stream>>>(p);
+        prepass_stats_kernel<128><<<gs, 256, ks_smem, stream>>>(p);
     else
-        prepass_stats_kernel<64><<<gs, 256, 0, stream>>>(p);
+        prepass_stats_kernel<64><<<gs, 256, ks_smem, stream>>>(p);
     SA_CHECK_LAUNCH();
-    const unsigned gq = (unsigned)(3 * BH * T);
     const bool ss = mode == SA_SCALE_SEARCH, sm = p.smooth_k != 0;
-#define SA_PQ(DD, SS, SM) prepass_quant_kernel<DD, SS, SM><<<gq, 2 * DD, 0, stream>>>(p)
+    // persistent: as many CTAs as fit on the GPU, each double-buffering tiles
+#define SA_PQ(DD, SS, SM)                                                                                      \
+    do {                                                                                                       \
+        const int smem = (int)sizeof(PqSmem<DD>);                                                              \
+        static int per_sm = 0; /* set once, outside any stream capture */                                      \
+        if (!per_sm) {                                                                                         \
+            if (cudaFuncSetAttribute(prepass_quant_kernel<DD, SS, SM>,                                         \
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||      \
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prepass_quant_kernel<DD, SS, SM>, 2 * DD, \
+                                                              smem) != cudaSuccess || per_sm < 1)              \
+                return SA_ERR_CUDA;                                                                            \
+        }                                                                                                      \
+        const unsigned gq = (unsigned)std::min<long>(3L * BH * T, (long)per_sm * sm_count());                  \
+        prepass_quant_kernel<DD, SS, SM><<<gq, 2 * DD, smem, stream>>>(p);                                     \
+    } while (0)
     if (D == 128) {
         if (ss) { if (sm) SA_PQ(128, true, true); else SA_PQ(128, true, false); }
         else { if (sm) SA_PQ(128, false, true); else SA_PQ(128, false, false); }
