@@ -47,7 +47,7 @@ struct PpSmem {
     alignas(16) uint8_t qsf[2][2][D / 64 * 512];
     uint8_t ksf[kPpStages][D / 64 * 512];
     uint8_t vsf[kPpStages][2 * 512];
-    float lg2tab[16];  // log2 of E4M3 significands: [m] normal (1 + m/8), [8 + m] subnormal (m/4)
+    float lg2sc[128];  // log2 of each nonzero E4M3 scale value: exponent + log2 of the significand
     uint64_t q_full[2];   // [item % 2]: Q tiles and scale atoms landed
     uint64_t q_empty[2];  // [item % 2]: every Q K^T of the item completed
     uint64_t kv_full[kPpStages];
@@ -179,7 +179,12 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    if (tid < 16) s.lg2tab[tid] = tid < 8 ? log2f(1.0f + tid * 0.125f) : log2f((tid - 8) * 0.25f);
+    if (tid < 128) {
+        // (e - 7) + log2(1 + m/8) for normal bytes, -7 + log2(m/4) for subnormal ones
+        const uint32_t e = (uint32_t)tid >> 3, m = (uint32_t)tid & 7u;
+        const float sig = e ? log2f(1.0f + m * 0.125f) : log2f(m * 0.25f);
+        s.lg2sc[tid] = (e ? (float)((int)e - 7) : -7.0f) + sig;
+    }
     // rows D..127 of every V stage are zero, rows 128..143 are E2M1 1.0
     for (int i = tid; i < kPpStages * (144 - D) * 16; i += blockDim.x) {
         const int st = i / ((144 - D) * 16), w = i % ((144 - D) * 16);
@@ -384,15 +389,19 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 float bias[8];
                 uint32_t scw0 = 0, scw1 = 0;
 #pragma unroll
-                for (int blk = 0; blk < 8; blk++) {
-                    const uint32_t sc = f32_to_e4m3(ex2f(fmaf(bmax[blk], c2, lm)) * (1.0f / 6.0f));
-                    const uint32_t e = sc >> 3, m = sc & 7u;
-                    const float lg2s = (e ? (float)((int)e - 7) : -7.0f) + s.lg2tab[(e ? 0u : 8u) + m];
-                    bias[blk] = sc ? lm - lg2s : -INFINITY;
-                    if (blk < 4)
-                        scw0 |= sc << (8 * blk);
-                    else
-                        scw1 |= sc << (8 * (blk - 4));
+                for (int bp = 0; bp < 8; bp += 2) {
+                    const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
+                                                         ex2f(fmaf(bmax[bp + 1], c2, lm)) * (1.0f / 6.0f));
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int blk = bp + h;
+                        const uint32_t sc = (sc2 >> (8 * h)) & 0xFFu;
+                        bias[blk] = sc ? lm - s.lg2sc[sc] : -INFINITY;
+                        if (blk < 4)
+                            scw0 |= sc << (8 * blk);
+                        else
+                            scw1 |= sc << (8 * (blk - 4));
+                    }
                 }
                 // y = P * 2688 / scale, rounded to E2M1
                 uint32_t codes[16];

@@ -42,6 +42,15 @@ SA_DEV uint32_t f32_to_e4m3(float x)
     return r & 0xFFu;
 }
 
+// Two non-negative finite floats -> two E4M3 bytes (a in the low byte), each
+// rounded and saturated as f32_to_e4m3 does, in one conversion.
+SA_DEV uint32_t f32x2_to_e4m3x2(float a, float b)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+    return r;
+}
+
 // Eight floats -> eight E2M1 nibbles (round to nearest even, saturating to
 // +-6, sign kept), element 0 in the lowest nibble.
 SA_DEV uint32_t pack8_e2m1(float y0, float y1, float y2, float y3, float y4, float y5, float y6, float y7)

@@ -494,17 +494,19 @@ __global__ void __launch_bounds__(2 * D) quant_v_kernel(const uint16_t* __restri
 // Fused pre-pass of Q, K and V (one statistics launch, one quantisation launch)
 // ---------------------------------------------------------------------------
 
-// max over the uint4 groups i0 + u stride (u < kAmaxPer) of the bf16
-// magnitude bits (|x| order == unsigned order of bits & 0x7FFF); all loads
-// are issued before the first use.  Normal (L2-keeping) loads: the
-// quantisation pass reads the same bytes next.
+// max over the uint4 groups base + tid + 256 u (u < kAmaxPer) of the bf16
+// magnitude bits (|x| order == unsigned order of bits & 0x7FFF): a block
+// reads one contiguous 32 KB chunk, so the blocks in flight cover one
+// contiguous range and spread over all HBM channels.  All loads are issued
+// before the first use.  Normal (L2-keeping) loads: the quantisation pass
+// reads the same bytes next.
 constexpr int kAmaxPer = 8;
-SA_DEV uint32_t amax_bits_batch(const uint4* __restrict__ x, size_t n16, size_t i0, size_t stride)
+SA_DEV uint32_t amax_bits_batch(const uint4* __restrict__ x, size_t n16, size_t base, int tid)
 {
     uint4 v[kAmaxPer];
 #pragma unroll
     for (int u = 0; u < kAmaxPer; u++) {
-        const size_t i = i0 + u * stride;
+        const size_t i = base + tid + 256 * u;
         v[u] = i < n16 ? __ldg(x + i) : make_uint4(0, 0, 0, 0);
     }
     uint32_t m = 0;
@@ -593,8 +595,8 @@ __global__ void __launch_bounds__(256) prepass_stats_kernel(const PrepassParams 
         const int which = a < p.nA ? 0 : (a < 2 * p.nA ? 2 : 1);
         const uint4* x = which == 0 ? p.q : (which == 2 ? p.v : p.k);
         const int lb = a - (which == 0 ? 0 : (which == 2 ? p.nA : 2 * p.nA));
-        // nA * 256 * kAmaxPer >= n16: one batch covers the tensor
-        uint32_t mm = amax_bits_batch(x, n16, (size_t)lb * blockDim.x + tid, (size_t)p.nA * blockDim.x);
+        // nA * 256 * kAmaxPer >= n16: one batch per block covers the tensor
+        uint32_t mm = amax_bits_batch(x, n16, (size_t)lb * 256 * kAmaxPer, tid);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mm = max(mm, __shfl_xor_sync(0xffffffffu, mm, o));
         if ((tid & 31) == 0) red[tid >> 5] = mm;
