@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 256 << 20
 # batch: each NVFP4 code and scale byte is read once).  Keyed by workload and
 # kernel; any other pair reports null.
 MEASURED_TRAFFIC = {
-    ("llm", "attn_fwd_pp_kernel<128>"): 14.49e6 * 2,  # B1 slice x 2
+    ("llm", "attn_fwd_pp_kernel<128>"): 14.74e6 * 2,  # B1 slice x 2
     ("decode", "decode_kernel<128> + combine"): 306.0e6 * 4,  # B8 slice x 4
 }
 
