@@ -129,12 +129,17 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
  * Same operation, arguments and bit-identical outputs as calling
  * sa_quant_nvfp4 for role Q (smooth 0), K (smooth = smooth_k) and V with the
  * same mode and offsets; no ScaleSearch offset outputs.
- *  q_dev, k_dev, v_dev   bf16 [B,H,N,D] inputs.
- *  *_codes, *_scales, *_g   outputs as sa_quant_nvfp4 for each role.
+ *  q_dev, k_dev, v_dev   bf16 [B,H,N,D] inputs, 16-byte aligned.
+ *  *_codes, *_scales, *_g   outputs as sa_quant_nvfp4 for each role (codes
+ *              8-byte aligned).
  *  k_mean_dev  float [B,H,D] channel means of K (written when smooth_k), may
  *              be NULL.
  *  ws_dev      scratch of sa_quant_qkv_workspace_size() bytes (256-byte
- *              aligned).
+ *              aligned); the call resets the part it needs with one
+ *              cudaMemsetAsync on the stream.
+ * Both kernels are persistent-style streams over 128-row tiles; the first
+ * call in a process also sets their shared-memory attributes (no stream
+ * work), so it may be made inside a stream capture or before one.
  * Errors: as sa_quant_nvfp4 (argument errors before any launch; non-finite
  * input in any of the three tensors -> SA_ERR_NONFINITE in the status word).
  * ------------------------------------------------------------------------ */
