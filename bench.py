@@ -259,6 +259,22 @@ def cpu_baseline(w, mode, budget_s=20.0):
                       f"{len(rows_done)}/{T} query tiles of all {B * H} heads ({t_attn:.1f} s)"}
 
 
+def max_over_ranks(values, pg, device):
+    """Element-wise max over all ranks of a list of floats (per-rank device
+    timings); the values themselves on a single rank."""
+    if pg is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tops(world, flops_per_rank, ms_max):
+    """Weak scaling: every rank runs the full workload, so the job's work is
+    world x the per-rank FLOPs, over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def run_reference(args, w, rank, world):
     if rank != 0:
         return
@@ -362,10 +378,7 @@ def main():
     assert st == 0, sa.STATUS[st]
     ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
     ms_attn = sum(a.elapsed_time(b) for a, b in aevs) / args.steps
-    if pg:
-        t = torch.tensor([ms, ms_attn], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms, ms_attn = t.tolist()
+    ms, ms_attn = max_over_ranks([ms, ms_attn], pg, dev)
 
     # end to end through the C ABI from pinned host buffers: copy the step's
     # inputs in, run the path, copy the output back
@@ -388,11 +401,7 @@ def main():
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e = statistics.mean(e2e_ms)
-    if pg:
-        t = torch.tensor([e2e], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e = t.item()
+    (e2e,) = max_over_ranks([statistics.mean(e2e_ms)], pg, dev)
     h2d_bytes = sum(src.numel() * src.element_size() for _, src in h2d)
 
     if rank == 0:
@@ -415,12 +424,12 @@ def main():
                     "traffic": traffic_of(w, kname, args), "traffic_unit": "bytes per launch (ncu, batch slice scaled)",
                     "ms_per_launch": ms_attn}
         line = {
-            "metric": METRIC, "value": world * flops / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world,
+            "metric": METRIC, "value": whole_job_tops(world, flops, ms), "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
             "config": config_of(w, args.mode),
             "roofline": roof,
-            "e2e": {"value": world * flops / (e2e * 1e-3) / 1e12, "unit": "TOPS",
+            "e2e": {"value": whole_job_tops(world, flops, e2e), "unit": "TOPS",
                     "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": hout.numel() * 4},
             "gpu_launches": kernels_per_step(w) * args.steps,
             "clocks": clk.summary(),
