@@ -43,7 +43,7 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel; any other pair reports null.
 MEASURED_TRAFFIC = {
     ("llm", "attn_fwd_pp_kernel<128>"): 14.74e6 * 2,  # B1 slice x 2
-    ("decode", "decode_kernel<128> + combine"): 306.0e6 * 4,  # B8 slice x 4
+    ("decode", "decode_kernel<128> + combine"): 305.7e6 * 4,  # B8 slice x 4
 }
 
 
