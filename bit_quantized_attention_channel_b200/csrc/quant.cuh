@@ -7,15 +7,22 @@
 // "SageAttention" (hotpaper.ai), "기술적 접근법": K minus its per-channel
 // mean over tokens.
 //
-// Kernels (all HBM-streaming, 16-byte loads where the layout allows):
-//   amax_bf16_kernel   max |x| over a tensor on the bf16 bit patterns
-//                      (|x| order == unsigned order of (bits & 0x7FFF)).
-//   kstats_kernel      per (b,h,128-token tile, channel): FP64 sum in token
-//                      order, max, min.
-//   kfinal_kernel      per (b,h,channel): tile partials in tile order -> mean;
-//                      amax of K - mean from max/min (rounding is monotone).
-//   quant_rows_kernel  Q/K: one thread per 16-channel block.
-//   quant_v_kernel     V: one thread per 16-token block of four channels.
+// Kernels (all HBM-streaming; tiles move by 16-byte loads or bulk copies):
+//   Per tensor (sa_quant_nvfp4):
+//   amax_bf16_kernel      max |x| over a tensor on the bf16 bit patterns
+//                         (|x| order == unsigned order of (bits & 0x7FFF)).
+//   kstats_kernel         per (b,h,128-token tile, channel): FP64 sum in
+//                         token order, max, min.
+//   kfinal_kernel         per (b,h,channel): tile partials in tile order ->
+//                         mean; amax of K - mean from max/min (rounding is
+//                         monotone).
+//   quant_rows_kernel     Q/K: one CTA per 128-row tile, one bulk copy.
+//   quant_v_kernel        V: one CTA per 128-token tile, one bulk copy.
+//   Q, K and V together (sa_quant_nvfp4_qkv), the same bytes:
+//   prepass_stats_kernel  K tiles (statistics, ticketed final reduction),
+//                         then the Q and V amax.
+//   prepass_quant_kernel  persistent; V, Q, K tiles double-buffered in
+//                         shared memory.
 #pragma once
 
 #include "common.cuh"
