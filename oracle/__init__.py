@@ -59,6 +59,8 @@ def lib():
         L.orc_attn_f64.restype = i
         L.orc_decode_f64.argtypes = [P, P, P, i, i, i, i, i, d, i, i, P, i, P]
         L.orc_decode_f64.restype = i
+        L.orc_decode_sink_f64.argtypes = [P, P, P, i, i, i, i, i, d, i, i, i, i, P, P, P, P, i, P]
+        L.orc_decode_sink_f64.restype = i
         L.orc_thrift_select.argtypes = [P, P, i, i, i, i, i, i, P, P, P]
         L.orc_thrift_select.restype = i
         L.orc_num_threads.restype = i
@@ -230,31 +232,54 @@ def attention(qq: Quantized, kq: Quantized, vq: Quantized, causal: bool, sm_scal
     return attn_f64(q, k, v, causal, sm_scale, True, mask, q_raw, k_s, v_raw, rows, want_lse)
 
 
-def decode_f64(q, k, v, sm_scale: float, quant_p: bool = True, split: int = 4096, pairs=None):
-    """Split-KV decode on FP64 operands: q [B,Hq,D], k/v [B,Hkv,L,D]."""
+def decode_f64(q, k, v, sm_scale: float, quant_p: bool = True, split: int = 4096, pairs=None,
+               sink_tiles=(0, 0), q_raw=None, k_raw_smoothed=None, v_raw=None):
+    """Split-KV decode on FP64 operands: q [B,Hq,D], k/v [B,Hkv,L,D].
+    sink_tiles = (first, last): that many 128-key tiles at each end of the
+    cache use the raw operands (q_raw [B,Hq,D], k_raw_smoothed and v_raw
+    [B,Hkv,L,D]) with bf16-rounded P."""
     q, k, v = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v))
     B, Hq, D = q.shape
     _, Hkv, L, _ = k.shape
     pp = None if pairs is None else np.ascontiguousarray(pairs, dtype=np.int32)
     npairs = B * Hq if pp is None else len(pp)
     out = np.zeros((npairs, D), np.float64)
-    rc = lib().orc_decode_f64(_p(q), _p(k), _p(v), B, Hq, Hkv, L, D, float(sm_scale), int(quant_p), int(split),
-                              _p(pp), npairs, _p(out))
+    first, last = (int(t) for t in sink_tiles)
+    if first or last:
+        q_raw, k_raw_smoothed, v_raw = (np.ascontiguousarray(a, dtype=np.float64) for a in
+                                        (q_raw, k_raw_smoothed, v_raw))
+        assert q_raw.shape == q.shape and k_raw_smoothed.shape == k.shape and v_raw.shape == v.shape
+    else:
+        q_raw = k_raw_smoothed = v_raw = None
+    rc = lib().orc_decode_sink_f64(_p(q), _p(k), _p(v), B, Hq, Hkv, L, D, float(sm_scale), int(quant_p), int(split),
+                                   first, last, _p(q_raw), _p(k_raw_smoothed), _p(v_raw), _p(pp), npairs, _p(out))
     if rc != 0:
-        raise ValueError(f"orc_decode_f64 failed: {rc}")
+        raise ValueError(f"orc_decode_sink_f64 failed: {rc}")
     return out
 
 
-def decode(q_bf16, kq: Quantized, vq: Quantized, sm_scale: float | None = None, split: int = 4096, pairs=None):
+def decode(q_bf16, kq: Quantized, vq: Quantized, sm_scale: float | None = None, split: int = 4096, pairs=None,
+           sink_tiles=(0, 0), k_bf16=None, v_bf16=None):
     """NVFP4-KV decode: q [B,Hq,D] bf16 is quantised like a Q tensor (its own
-    per-tensor scale, blocks along D, max-scaling)."""
+    per-tensor scale, blocks along D, max-scaling).  sink_tiles = (first,
+    last) keeps that many 128-key tiles at each end of the cache at full
+    precision ("ScaleSearchAttention", attention-sink-aware mixed-precision
+    caching); they need the raw bf16 cache k_bf16, v_bf16 [B,Hkv,L,D], and
+    the smoothed K mean of kq offsets their keys like the NVFP4 ones."""
     qb = bf16_bits(q_bf16)
     B, Hq, D = qb.shape
     qq = quantize(qb.reshape(1, B, Hq, D), "q", smooth=False, search=False)
     qd = qq.dequant().reshape(B, Hq, D)
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(D)
-    return decode_f64(qd, kq.dequant(), vq.dequant(), sm_scale, True, split, pairs)
+    q_raw = k_s = v_raw = None
+    if sink_tiles[0] or sink_tiles[1]:
+        q_raw = bf16_to_f64(qb)
+        k_s = bf16_to_f64(bf16_bits(k_bf16))
+        if kq.k_mean is not None:
+            k_s = k_s - kq.k_mean.astype(np.float64)[:, :, None, :]
+        v_raw = bf16_to_f64(bf16_bits(v_bf16))
+    return decode_f64(qd, kq.dequant(), vq.dequant(), sm_scale, True, split, pairs, sink_tiles, q_raw, k_s, v_raw)
 
 
 # ---------------------------------------------------------------- selector

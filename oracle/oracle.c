@@ -44,7 +44,11 @@
  *    max-scaling; the denominator l sums the dequantised P;
  *  - the selector mean-pools 128-row tiles of raw Q and K into bf16, scores
  *    with an FP32 fmaf chain, and keeps the top ceil(frac * valid) blocks per
- *    head, ties broken by the lower block index.
+ *    head, ties broken by the lower block index;
+ *  - the attention-sink-aware decode cache keeps whole 128-key tiles at full
+ *    precision: a count of tiles at the start and at the end of the cache,
+ *    with the raw bf16 operands, bf16-rounded P and the smoothed keys' mean
+ *    offset, as the mixed blocks of the prefill schedule do.
  */
 #include <math.h>
 #include <stdint.h>
@@ -514,31 +518,55 @@ int orc_attn_f64(const double* q, const double* k, const double* v, long BH, int
  *   O = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s,  M = max_s m_s.
  * q: [B, Hq, D] FP64 (already quantised/dequantised), k, v: [B, Hkv, L, D].
  * pairs/npairs: (b, hq) flat indices to compute (NULL = all); out [npairs, D].
+ *
+ * Attention-sink-aware mixed-precision cache [SS "ScaleSearchAttention",
+ * attention-sink-aware mixed-precision caching]: the first sink_first and the
+ * last sink_last 128-key tiles of the cache are kept at full precision and the
+ * rest in NVFP4.  Those tiles take the mixed-block arithmetic of attn_row:
+ * raw bf16 q (q_raw [B, Hq, D]), raw bf16 k minus its channel mean
+ * (k_raw_smoothed [B, Hkv, L, D]), bf16-rounded P and raw bf16 v (v_raw), in
+ * the same split-wise online softmax.  sink_first = sink_last = 0 is the plain
+ * NVFP4 decode and needs no raw operands.
  */
-int orc_decode_f64(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int L, int D,
-                   double sm_scale, int quant_p, int split, const int32_t* pairs, int npairs, double* out)
+int orc_decode_sink_f64(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int L, int D,
+                        double sm_scale, int quant_p, int split, int sink_first, int sink_last, const double* q_raw,
+                        const double* k_raw_smoothed, const double* v_raw, const int32_t* pairs, int npairs,
+                        double* out)
 {
     init_formats();
     if (Hkv <= 0 || Hq % Hkv || L <= 0 || split <= 0 || split % TILE) return -1;
+    if (sink_first < 0 || sink_last < 0) return -1;
+    const int mixed = sink_first > 0 || sink_last > 0;
+    if (mixed && (!q_raw || !k_raw_smoothed || !v_raw)) return -1;
     int grp = Hq / Hkv;
     int np = pairs ? npairs : B * Hq;
     int nsplit = (L + split - 1) / split;
+    int T = (L + TILE - 1) / TILE;  /* key tiles of the whole cache */
 #pragma omp parallel for schedule(dynamic, 1)
     for (int pi = 0; pi < np; pi++) {
         int flat = pairs ? pairs[pi] : pi;
         int b = flat / Hq, hq = flat % Hq, hk = hq / grp;
+        size_t kvo = ((size_t)b * Hkv + hk) * L * D;
         const double* qr = q + (size_t)flat * D;
-        const double* kb = k + ((size_t)b * Hkv + hk) * L * D;
-        const double* vb = v + ((size_t)b * Hkv + hk) * L * D;
+        const double* kb = k + kvo;
+        const double* vb = v + kvo;
         double* ms = (double*)malloc(sizeof(double) * nsplit);
         double* ls = (double*)malloc(sizeof(double) * nsplit);
         double* os = (double*)malloc(sizeof(double) * nsplit * D);
+        uint8_t* flags = (uint8_t*)malloc((size_t)split / TILE);
         double M = -INFINITY;
         for (int s = 0; s < nsplit; s++) {
             int k0 = s * split;
             int n = L - k0 < split ? L - k0 : split;
-            attn_row(qr, kb + (size_t)k0 * D, vb + (size_t)k0 * D, n, D, -1, sm_scale, quant_p, NULL, NULL, NULL,
-                     NULL, &ms[s], &ls[s], os + (size_t)s * D);
+            int nt = (n + TILE - 1) / TILE;
+            for (int u = 0; u < nt; u++) {
+                int g = k0 / TILE + u; /* tile index in the cache */
+                flags[u] = (uint8_t)(g < sink_first || g >= T - sink_last);
+            }
+            attn_row(qr, kb + (size_t)k0 * D, vb + (size_t)k0 * D, n, D, -1, sm_scale, quant_p,
+                     mixed ? flags : NULL, mixed ? q_raw + (size_t)flat * D : NULL,
+                     mixed ? k_raw_smoothed + kvo + (size_t)k0 * D : NULL, mixed ? v_raw + kvo + (size_t)k0 * D : NULL,
+                     &ms[s], &ls[s], os + (size_t)s * D);
             if (ms[s] > M) M = ms[s];
         }
         double den = 0.0;
@@ -553,8 +581,17 @@ int orc_decode_f64(const double* q, const double* k, const double* v, int B, int
         free(ms);
         free(ls);
         free(os);
+        free(flags);
     }
     return 0;
+}
+
+/* The plain NVFP4-KV decode: no full-precision tiles. */
+int orc_decode_f64(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int L, int D,
+                   double sm_scale, int quant_p, int split, const int32_t* pairs, int npairs, double* out)
+{
+    return orc_decode_sink_f64(q, k, v, B, Hq, Hkv, L, D, sm_scale, quant_p, split, 0, 0, NULL, NULL, NULL, pairs,
+                               npairs, out);
 }
 
 /* ------------------------------------------------------------------------ */

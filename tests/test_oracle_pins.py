@@ -428,6 +428,117 @@ def test_decode_quantized_convex():
         assert np.all(out[:, hq] >= lo - 1e-12) and np.all(out[:, hq] <= hi + 1e-12)
 
 
+# ------------------------------------------------ sink-aware mixed-precision decode
+def _exact_decode(q, k, v, sm):
+    """Exact FP64 decode on raw operands: q [B,Hq,D], k/v [B,Hkv,L,D]."""
+    B, Hq, D = q.shape
+    grp = Hq // k.shape[1]
+    kk, vv = np.repeat(k, grp, axis=1), np.repeat(v, grp, axis=1)
+    return _exact_attention(q[:, :, None, :], kk, vv, False, sm)[:, :, 0, :].reshape(B * Hq, D)
+
+
+def _sink_case(L=1024, D=64, alpha=1.0, seed=11):
+    """A cache whose score mass sits in its first and last 128-key tiles:
+    those keys are alpha * q of their query group plus noise, the rest are
+    noise (scores ~ 8 alpha against ~ N(0, 1) at sm_scale 1/sqrt(D))."""
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv = 1, 4, 2
+    q = rng.standard_normal((B, Hq, D))
+    k = rng.standard_normal((B, Hkv, L, D))
+    for hk in range(Hkv):
+        qm = q[:, 2 * hk: 2 * hk + 2].mean(1)  # both query heads of the group
+        for lo, hi in ((0, 128), (L - 128, L)):
+            k[:, hk, lo:hi] = alpha * qm[:, None, :] + 0.3 * rng.standard_normal((B, hi - lo, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    return tuple(torch.from_numpy(a).to(torch.bfloat16) for a in (q, k, v))
+
+
+def test_decode_sink_none_is_plain_decode():
+    q, k, v = wl.decode_inputs(B=1, Hq=4, Hkv=2, L=512, D=64)
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    a = orc.decode(q, kq, vq, split=256)
+    b = orc.decode(q, kq, vq, split=256, sink_tiles=(0, 0), k_bf16=k, v_bf16=v)
+    assert np.array_equal(a, b)
+
+
+def test_decode_sink_all_tiles_is_exact_up_to_bf16_p():
+    """Every tile at full precision: exact attention on the raw bf16 cache
+    (the K channel mean cancels in the softmax), up to the bf16 rounding of
+    P (relative 2^-8 per weight).  Which end the full-precision tiles are
+    counted from does not matter."""
+    q, k, v = wl.decode_inputs(B=2, Hq=4, Hkv=2, L=1024, D=64)
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    T = 1024 // 128
+    a = orc.decode(q, kq, vq, split=256, sink_tiles=(T, 0), k_bf16=k, v_bf16=v)
+    b = orc.decode(q, kq, vq, split=256, sink_tiles=(3, T - 3), k_bf16=k, v_bf16=v)
+    assert np.array_equal(a, b)
+    ref = _exact_decode(q.double().numpy(), k.double().numpy(), v.double().numpy(), 1 / 8)
+    assert np.max(np.abs(a - ref)) <= 2.0 ** -7 * np.max(np.abs(v.double().numpy()))
+
+
+def test_decode_sink_tiles_carry_the_attention_mass():
+    """Scores concentrated on the first and last tiles (an attention sink and
+    the recent tokens): keeping those two tiles at full precision brings the
+    output to the bf16-P error of exact attention, far below the error of the
+    all-NVFP4 cache ("ScaleSearchAttention", attention-sink-aware
+    mixed-precision caching)."""
+    q, k, v = _sink_case()
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    ref = _exact_decode(q.double().numpy(), k.double().numpy(), v.double().numpy(), 1 / 8)
+    vmax = np.max(np.abs(v.double().numpy()))
+    fp4 = orc.decode(q, kq, vq, split=256)
+    sink = orc.decode(q, kq, vq, split=256, sink_tiles=(1, 1), k_bf16=k, v_bf16=v)
+    err_fp4, err_sink = np.max(np.abs(fp4 - ref)), np.max(np.abs(sink - ref))
+    assert err_sink <= 2.0 ** -7 * vmax
+    assert err_sink < err_fp4 / 4
+
+
+def test_decode_sink_output_is_convex():
+    """Each output column lies between the smallest and largest value it
+    averages: dequantised V in the NVFP4 tiles, raw V in the sink tiles."""
+    q, k, v = wl.decode_inputs(B=2, Hq=4, Hkv=2, L=768, D=64)
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    out = orc.decode(q, kq, vq, split=256, sink_tiles=(1, 2), k_bf16=k, v_bf16=v).reshape(2, 4, 64)
+    V, Vr = vq.dequant(), v.double().numpy()
+    for hq in range(4):
+        hk = hq // 2
+        vals = np.concatenate([V[:, hk, 128:768 - 256], Vr[:, hk, :128], Vr[:, hk, 768 - 256:]], axis=1)
+        lo, hi = vals.min(1), vals.max(1)
+        assert np.all(out[:, hq] >= lo - 1e-12) and np.all(out[:, hq] <= hi + 1e-12)
+
+
+def test_decode_sink_keys_share_the_fp4_score_offset():
+    """With a strong per-channel K offset (scores shift by q.mu), the
+    full-precision tiles must subtract the same channel mean as the smoothed
+    NVFP4 tiles; otherwise their scores would move by q.mu * sm_scale
+    (several units here) against the rest and the output would be far off."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, L, D = 1, 4, 2, 768, 64
+    q = rng.standard_normal((B, Hq, D))
+    k = rng.standard_normal((B, Hkv, L, D)) + 3.0 * rng.standard_normal((B, Hkv, 1, D))
+    v = rng.standard_normal((B, Hkv, L, D))
+    q, k, v = (torch.from_numpy(a).to(torch.bfloat16) for a in (q, k, v))
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    ref = _exact_decode(q.double().numpy(), k.double().numpy(), v.double().numpy(), 1 / 8)
+    err_fp4 = np.max(np.abs(orc.decode(q, kq, vq, split=256) - ref))
+    sink = orc.decode(q, kq, vq, split=256, sink_tiles=(2, 2), k_bf16=k, v_bf16=v)
+    assert np.max(np.abs(sink - ref)) <= err_fp4
+
+
+def test_decode_sink_rejects_bad_arguments():
+    q, k, v = wl.decode_inputs(B=1, Hq=2, Hkv=1, L=256, D=32)
+    kq, vq = orc.quantize(k, "k"), orc.quantize(v, "v")
+    qd = orc.bf16_to_f64(orc.bf16_bits(q))
+    K, V = kq.dequant(), vq.dequant()
+    with pytest.raises(ValueError):
+        orc.decode_f64(qd, K, V, 0.1, sink_tiles=(-1, 0), q_raw=qd, k_raw_smoothed=K, v_raw=V)
+    # the full-precision tiles need the raw operands: NULLs are rejected
+    out = np.zeros((2, 32))
+    rc = orc.lib().orc_decode_sink_f64(orc._p(qd), orc._p(K), orc._p(V), 1, 2, 1, 256, 32, 0.1, 1, 256, 1, 0, None,
+                                       None, None, None, 2, orc._p(out))
+    assert rc == -1
+
+
 # ------------------------------------------------------------------ selector
 def test_selector_scores_count_topk_and_validity():
     q, k, _ = wl.prefill_inputs("longctx", B=1, H=2, N=1024, D=64)
