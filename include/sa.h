@@ -137,9 +137,10 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
  *  ws_dev      scratch of sa_quant_qkv_workspace_size() bytes (256-byte
  *              aligned); the call resets the part it needs with one
  *              cudaMemsetAsync on the stream.
- * Both kernels are persistent-style streams over 128-row tiles; the first
- * call in a process also sets their shared-memory attributes (no stream
- * work), so it may be made inside a stream capture or before one.
+ * The quantisation kernel is persistent over 128-row tiles.  The first call
+ * in a process also sets its shared-memory attribute and reads its occupancy
+ * (host-side, no stream work); make that first call outside any stream
+ * capture (later calls may be captured into a CUDA graph).
  * Errors: as sa_quant_nvfp4 (argument errors before any launch; non-finite
  * input in any of the three tensors -> SA_ERR_NONFINITE in the status word).
  * ------------------------------------------------------------------------ */
