@@ -226,6 +226,7 @@ ATTN_CASES = [
     ("tiny", {"N": 640, "D": 128}, True, "max", None),  # odd tile count: last CTA has one query tile
     ("llm", {}, True, "max", "sample"),
     ("llm", {}, True, "search", "sample"),
+    ("video", {}, False, "search", "sample"),         # full video size: non-causal, ~21 items per CTA
 ]
 
 
