@@ -67,6 +67,7 @@ def lib():
         L.orc_quant_block.argtypes = [P, i, i, i, P, P, P, P]
         L.orc_block_err.argtypes, L.orc_block_err.restype = [P, i], f
         L.orc_requant_p.argtypes = [P, i, P]
+        L.orc_requant_p_mode.argtypes, L.orc_requant_p_mode.restype = [P, i, P, i], i
         _lib = L
     return _lib
 
@@ -123,6 +124,22 @@ def requant_p(pt):
     out = np.zeros_like(p)
     lib().orc_requant_p(_p(p), len(p), _p(out))
     return out
+
+
+def requant_p_search(pt, search: bool = True):
+    """One block of P~ (at most 16 values) requantised with ScaleSearch (or
+    max-scaling): (dequantised P^, chosen E4M3 scale code)."""
+    p = np.ascontiguousarray(pt, dtype=np.float64)
+    out = np.zeros_like(p)
+    c = lib().orc_requant_p_mode(_p(p), len(p), _p(out), int(search))
+    return out, c
+
+
+def _quant_p_mode(quant_p, p_search: bool) -> int:
+    """0: P~ kept unquantised, 1: max-scaling, 2: ScaleSearch on P."""
+    if not quant_p:
+        return 0
+    return 2 if p_search else 1
 
 
 def tensor_scale(amax: float):
@@ -194,9 +211,10 @@ def quantize(x, role: str, smooth: bool = True, search: bool = False, f_lo: int 
 
 # ---------------------------------------------------------------- attention
 def attn_f64(q, k, v, causal: bool, sm_scale: float, quant_p: bool = True, mask=None, q_raw=None,
-             k_raw_smoothed=None, v_raw=None, rows=None, want_lse: bool = False):
+             k_raw_smoothed=None, v_raw=None, rows=None, want_lse: bool = False, p_search: bool = False):
     """Run the attention schedule on FP64 [B,H,N,D] operands.  rows: optional
-    array of query-row indices (same for every head)."""
+    array of query-row indices (same for every head).  p_search: requantise
+    P with ScaleSearch instead of max-scaling."""
     q, k, v = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v))
     B, H, N, D = q.shape
     rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
@@ -207,7 +225,8 @@ def attn_f64(q, k, v, causal: bool, sm_scale: float, quant_p: bool = True, mask=
         mask = np.ascontiguousarray(mask, dtype=np.uint8)
         q_raw, k_raw_smoothed, v_raw = (np.ascontiguousarray(a, dtype=np.float64) for a in
                                         (q_raw, k_raw_smoothed, v_raw))
-    rc = lib().orc_attn_f64(_p(q), _p(k), _p(v), B * H, N, D, int(causal), float(sm_scale), int(quant_p), _p(mask),
+    rc = lib().orc_attn_f64(_p(q), _p(k), _p(v), B * H, N, D, int(causal), float(sm_scale),
+                            _quant_p_mode(quant_p, p_search), _p(mask),
                             _p(q_raw), _p(k_raw_smoothed), _p(v_raw), _p(rr), nr, _p(out), _p(lse))
     if rc != 0:
         raise ValueError(f"orc_attn_f64 failed: {rc}")
@@ -215,9 +234,10 @@ def attn_f64(q, k, v, causal: bool, sm_scale: float, quant_p: bool = True, mask=
 
 
 def attention(qq: Quantized, kq: Quantized, vq: Quantized, causal: bool, sm_scale: float | None = None, rows=None,
-              mask=None, q_bf16=None, k_bf16=None, v_bf16=None, want_lse: bool = False):
+              mask=None, q_bf16=None, k_bf16=None, v_bf16=None, want_lse: bool = False, p_search: bool = False):
     """NVFP4 attention forward on quantised operands (optionally with
-    high-precision blocks from `mask`, which then needs the raw bf16 inputs)."""
+    high-precision blocks from `mask`, which then needs the raw bf16 inputs).
+    p_search: ScaleSearch on the requantised P blocks."""
     B, H, N, D = qq.shape
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(D)
@@ -229,11 +249,11 @@ def attention(qq: Quantized, kq: Quantized, vq: Quantized, causal: bool, sm_scal
         if kq.k_mean is not None:
             k_s = k_s - kq.k_mean.astype(np.float64)[:, :, None, :]
         v_raw = bf16_to_f64(bf16_bits(v_bf16))
-    return attn_f64(q, k, v, causal, sm_scale, True, mask, q_raw, k_s, v_raw, rows, want_lse)
+    return attn_f64(q, k, v, causal, sm_scale, True, mask, q_raw, k_s, v_raw, rows, want_lse, p_search)
 
 
 def decode_f64(q, k, v, sm_scale: float, quant_p: bool = True, split: int = 4096, pairs=None,
-               sink_tiles=(0, 0), q_raw=None, k_raw_smoothed=None, v_raw=None):
+               sink_tiles=(0, 0), q_raw=None, k_raw_smoothed=None, v_raw=None, p_search: bool = False):
     """Split-KV decode on FP64 operands: q [B,Hq,D], k/v [B,Hkv,L,D].
     sink_tiles = (first, last): that many 128-key tiles at each end of the
     cache use the raw operands (q_raw [B,Hq,D], k_raw_smoothed and v_raw
@@ -251,7 +271,8 @@ def decode_f64(q, k, v, sm_scale: float, quant_p: bool = True, split: int = 4096
         assert q_raw.shape == q.shape and k_raw_smoothed.shape == k.shape and v_raw.shape == v.shape
     else:
         q_raw = k_raw_smoothed = v_raw = None
-    rc = lib().orc_decode_sink_f64(_p(q), _p(k), _p(v), B, Hq, Hkv, L, D, float(sm_scale), int(quant_p), int(split),
+    rc = lib().orc_decode_sink_f64(_p(q), _p(k), _p(v), B, Hq, Hkv, L, D, float(sm_scale),
+                                   _quant_p_mode(quant_p, p_search), int(split),
                                    first, last, _p(q_raw), _p(k_raw_smoothed), _p(v_raw), _p(pp), npairs, _p(out))
     if rc != 0:
         raise ValueError(f"orc_decode_sink_f64 failed: {rc}")

@@ -388,28 +388,22 @@ void orc_dequant(const uint8_t* codes, const uint8_t* scales, float g, size_t ro
 /* ------------------------------------------------------------------------ */
 
 /* One 16-key block of probabilities P~ (FP64, in [0,1]) to NVFP4 with the
- * fixed second-level scale 1/2688 and max-scaling; returns the dequantised
- * values P^ = E2M1 * E4M3 / 2688. */
-static void requant_p_block(const double* pt, int n, double* ph)
+ * fixed second-level scale 1/2688, i.e. the block of g-normalised values
+ * p~ = fl32(P~ * 2688) (a ragged tail is padded with zeros, which change
+ * neither the block max nor the error).  Max-scaling (search = 0) or
+ * ScaleSearch over the scale codes c0 + f, f in [-2, 6) (search = 1), as for
+ * Q, K and V [SS "메커니즘", "검색 전략"].  Returns the dequantised values
+ * P^ = E2M1 * E4M3 / 2688 and the chosen scale code. */
+static int requant_p_block(const double* pt, int n, double* ph, int search)
 {
     float pn[BLK];
-    float amax = 0.0f;
-    for (int i = 0; i < n; i++) {
-        pn[i] = (float)(pt[i] * 2688.0);
-        if (pn[i] > amax) amax = pn[i];
-    }
-    int c = orc_e4m3_code(amax / 6.0f);
-    if (c == 0) {
-        for (int i = 0; i < n; i++) ph[i] = 0.0;
-        return;
-    }
-    float s = (float)E4M3_MAG[c];
-    float r = 1.0f / s;
-    for (int i = 0; i < n; i++) {
-        float y = pn[i] * r;
-        int code = orc_e2m1_code(y);
-        ph[i] = orc_e2m1_value(code) * (double)s / 2688.0;
-    }
+    for (int i = 0; i < BLK; i++) pn[i] = i < n ? (float)(pt[i] * 2688.0) : 0.0f;
+    uint8_t code16[BLK], c;
+    int8_t off;
+    quant_block(pn, search, -2, 6, code16, &c, &off);
+    const double s = E4M3_MAG[c];
+    for (int i = 0; i < n; i++) ph[i] = c ? orc_e2m1_value(code16[i]) * s / 2688.0 : 0.0;
+    return c;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -422,7 +416,9 @@ static void requant_p_block(const double* pt, int n, double* ph)
  * masked (causal_limit < 0: none).  Mixed blocks [TA] use raw bf16 q and k
  * (k minus its channel mean, so FP4 and bf16 blocks share one score offset),
  * bf16-rounded P and raw V, inside the same running max / sum / output.
- * Returns m and l through the pointers; o receives the unnormalised sum. */
+ * quant_p: 0 keeps P~ unquantised, 1 requantises it with max-scaling, 2 with
+ * ScaleSearch.  Returns m and l through the pointers; o receives the
+ * unnormalised sum. */
 static void attn_row(const double* q, const double* kh, const double* vh, int nkeys, int D, long causal_limit,
                      double sm_scale, int quant_p, const uint8_t* mixed_tiles, const double* q_raw,
                      const double* k_raw_smoothed, const double* v_raw, double* m_out, double* l_out, double* o)
@@ -457,7 +453,7 @@ static void attn_row(const double* q, const double* kh, const double* vh, int nk
         } else if (quant_p) {
             for (int b0 = 0; b0 < n; b0 += BLK) {
                 int nb = n - b0 < BLK ? n - b0 : BLK;
-                requant_p_block(Pt + b0, nb, Ph + b0);
+                requant_p_block(Pt + b0, nb, Ph + b0, quant_p == 2);
             }
         } else {
             for (int jj = 0; jj < n; jj++) Ph[jj] = Pt[jj];
@@ -709,5 +705,13 @@ float orc_block_err(const float* xt, int c)
 void orc_requant_p(const double* pt, int n, double* ph)
 {
     init_formats();
-    requant_p_block(pt, n, ph);
+    requant_p_block(pt, n, ph, 0);
+}
+
+/* P requantisation of one block with max-scaling (search 0) or ScaleSearch
+ * (search 1); returns the chosen E4M3 scale code. */
+int orc_requant_p_mode(const double* pt, int n, double* ph, int search)
+{
+    init_formats();
+    return requant_p_block(pt, n, ph, search);
 }
