@@ -68,6 +68,10 @@ def lib():
         L.orc_block_err.argtypes, L.orc_block_err.restype = [P, i], f
         L.orc_requant_p.argtypes = [P, i, P]
         L.orc_requant_p_mode.argtypes, L.orc_requant_p_mode.restype = [P, i, P, i], i
+        L.orc_quant_rows_f32.argtypes = [P, ctypes.c_long, i, i, i, i, P, P, P, P]
+        L.orc_quant_rows_f32.restype = i
+        L.orc_incoherence.argtypes = [P, P, P, i, i, i, i, P, P, P, P]
+        L.orc_incoherence.restype = i
         _lib = L
     return _lib
 
@@ -207,6 +211,39 @@ def quantize(x, role: str, smooth: bool = True, search: bool = False, f_lo: int 
     if rc != 0:
         raise ValueError(f"orc_quant_nvfp4 failed: {rc}")
     return Quantized(codes, scales, float(g2[0]), float(g2[1]), kmean, off, role, (B, H, N, D))
+
+
+def quantize_rows_f32(x, search: bool = False, f_lo: int = -2, f_hi: int = 6) -> Quantized:
+    """Quantise FP32 [B,H,N,D] rows (Q/K block layout) to NVFP4 with the same
+    tensor scale and block rule as quantize(); no smoothing."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    B, H, N, D = x.shape
+    codes = np.zeros((B, H, N, D // 2), np.uint8)
+    scales = np.zeros((B, H, N, D // 16), np.uint8)
+    off = np.zeros(scales.shape, np.int8)
+    g2 = np.zeros(2, np.float32)
+    rc = lib().orc_quant_rows_f32(_p(x), B * H * N, D, int(search), f_lo, f_hi, _p(codes), _p(scales), _p(g2),
+                                  _p(off))
+    if rc != 0:
+        raise ValueError(f"orc_quant_rows_f32 failed: {rc}")
+    return Quantized(codes, scales, float(g2[0]), float(g2[1]), None, off, "q", (B, H, N, D))
+
+
+def incoherence(q_bf16, k_bf16, signs, k_mean=None):
+    """Incoherence processing of Q and K ("ScaleSearchAttention"): signed
+    Hadamard rotation and the per-(b,h,channel) balancing scale r.
+    Returns (Q' FP32, K' FP32, r FP32 [B,H,D])."""
+    qb, kb = bf16_bits(q_bf16), bf16_bits(k_bf16)
+    B, H, N, D = qb.shape
+    sg = np.ascontiguousarray(signs, dtype=np.int8)
+    km = None if k_mean is None else np.ascontiguousarray(k_mean, dtype=np.float32)
+    qo = np.zeros((B, H, N, D), np.float32)
+    ko = np.zeros((B, H, N, D), np.float32)
+    r = np.zeros((B, H, D), np.float32)
+    rc = lib().orc_incoherence(_p(qb), _p(kb), _p(km), B, H, N, D, _p(sg), _p(qo), _p(ko), _p(r))
+    if rc != 0:
+        raise ValueError(f"orc_incoherence failed: {rc}")
+    return qo, ko, r
 
 
 # ---------------------------------------------------------------- attention

@@ -45,6 +45,9 @@
  *  - the selector mean-pools 128-row tiles of raw Q and K into bf16, scores
  *    with an FP32 fmaf chain, and keeps the top ceil(frac * valid) blocks per
  *    head, ties broken by the lower block index;
+ *  - incoherence processing rotates Q and K by a signed Hadamard matrix and
+ *    balances each channel with a diagonal R (the minimiser of the summed
+ *    squared magnitudes), per (batch, head);
  *  - the attention-sink-aware decode cache keeps whole 128-key tiles at full
  *    precision: a count of tiles at the start and at the end of the cache,
  *    with the raw bf16 operands, bf16-rounded P and the smoothed keys' mean
@@ -363,6 +366,111 @@ int orc_quant_nvfp4(const uint16_t* x, int B, int H, int N, int D, int role, int
         }
     }
     free(mu);
+    return 0;
+}
+
+/*
+ * Quantise FP32 rows x[rows, D] (Q/K layout: blocks of 16 consecutive
+ * channels of a row) to NVFP4 with the same per-tensor scale and block rule
+ * as orc_quant_nvfp4 (no smoothing: the caller has applied any transform).
+ * Returns 0, -1 for bad arguments, -2 for non-finite input.
+ */
+int orc_quant_rows_f32(const float* x, long rows, int D, int search, int f_lo, int f_hi, uint8_t* codes,
+                       uint8_t* scales, float* g2, int8_t* ss_off)
+{
+    init_formats();
+    if (rows < 0 || D <= 0 || D % BLK) return -1;
+    size_t total = (size_t)rows * D;
+    float amax = 0.0f;
+    for (size_t i = 0; i < total; i++) {
+        if (!isfinite(x[i])) return -2;
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float g, inv_g;
+    orc_tensor_scale(amax, &g, &inv_g);
+    g2[0] = g;
+    g2[1] = inv_g;
+    int nb = D / BLK;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; r++) {
+        for (int b = 0; b < nb; b++) {
+            float xt[BLK];
+            uint8_t c16[BLK];
+            for (int i = 0; i < BLK; i++) xt[i] = x[(size_t)r * D + b * BLK + i] * inv_g;
+            uint8_t sc;
+            int8_t off;
+            quant_block(xt, search, f_lo, f_hi, c16, &sc, &off);
+            for (int i = 0; i < BLK / 2; i++)
+                codes[(size_t)r * (D / 2) + b * (BLK / 2) + i] =
+                    (uint8_t)((c16[2 * i] & 15) | ((c16[2 * i + 1] & 15) << 4));
+            scales[(size_t)r * nb + b] = sc;
+            if (ss_off) ss_off[(size_t)r * nb + b] = off;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Incoherence processing [SS "ScaleSearchAttention", "비일관성 처리 (IP) 및
+ * 크기 감소"]: a Hadamard transform of Q and K (following QuIP#: the
+ * orthonormal Sylvester matrix H_D, entries (-1)^popcount(i & j) / sqrt(D),
+ * followed by a diagonal of random signs S, given as input), then a linear
+ * pair Q' = Q~ R^-T, K' = K~ R that keeps every score Q' K'^T = Q~ K~^T and
+ * lowers the mean squared magnitude.  Reading: R is diagonal per (b, h,
+ * channel), the minimiser of |Q~ R^-1|^2 + |K~ R|^2 over diagonal R:
+ * r_c = (sum_t q~_tc^2 / sum_t k~_tc^2)^(1/4) (r_c = 1 when either sum is 0).
+ * Here Q~ = Q H S and K~ = (K - mu) H S, with mu the K channel mean (k_mean,
+ * nullable: no smoothing).  FP64 throughout; outputs rounded to FP32.
+ *  q, k: bf16 [B, H, N, D], D a power of two; signs: D entries of +-1.
+ *  q_out, k_out: FP32 [B, H, N, D]; r_out: FP32 [B, H, D].
+ */
+int orc_incoherence(const uint16_t* q, const uint16_t* k, const float* k_mean, int B, int H, int N, int D,
+                    const int8_t* signs, float* q_out, float* k_out, float* r_out)
+{
+    if (B < 0 || H < 0 || N <= 0 || D <= 0 || (D & (D - 1))) return -1;
+    for (int j = 0; j < D; j++)
+        if (signs[j] != 1 && signs[j] != -1) return -1;
+    const double hn = 1.0 / sqrt((double)D);
+    const long BH = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; bh++) {
+        double* yq = (double*)malloc(sizeof(double) * (size_t)N * D);
+        double* yk = (double*)malloc(sizeof(double) * (size_t)N * D);
+        double* x = (double*)malloc(sizeof(double) * D);
+        for (int t = 0; t < N; t++) {
+            for (int pass = 0; pass < 2; pass++) {
+                const uint16_t* src = (pass ? k : q) + ((size_t)bh * N + t) * D;
+                double* dst = (pass ? yk : yq) + (size_t)t * D;
+                for (int i = 0; i < D; i++) {
+                    float v = bf16_to_f32(src[i]);
+                    if (pass && k_mean) v = v - k_mean[(size_t)bh * D + i];
+                    x[i] = v;
+                }
+                for (int j = 0; j < D; j++) {  /* (x H)_j, then the sign of column j */
+                    double acc = 0.0;
+                    for (int i = 0; i < D; i++) acc += (__builtin_popcount((unsigned)(i & j)) & 1) ? -x[i] : x[i];
+                    dst[j] = acc * hn * signs[j];
+                }
+            }
+        }
+        for (int j = 0; j < D; j++) {
+            double a = 0.0, b = 0.0;
+            for (int t = 0; t < N; t++) {
+                a += yq[(size_t)t * D + j] * yq[(size_t)t * D + j];
+                b += yk[(size_t)t * D + j] * yk[(size_t)t * D + j];
+            }
+            double r = (a > 0.0 && b > 0.0) ? sqrt(sqrt(a / b)) : 1.0;
+            r_out[(size_t)bh * D + j] = (float)r;
+            for (int t = 0; t < N; t++) {
+                q_out[((size_t)bh * N + t) * D + j] = (float)(yq[(size_t)t * D + j] / r);
+                k_out[((size_t)bh * N + t) * D + j] = (float)(yk[(size_t)t * D + j] * r);
+            }
+        }
+        free(yq);
+        free(yk);
+        free(x);
+    }
     return 0;
 }
 

@@ -511,6 +511,73 @@ def test_decode_with_p_scalesearch_is_convex():
         assert np.all(out[:, hq] >= lo - 1e-12) and np.all(out[:, hq] <= hi + 1e-12)
 
 
+# ------------------------------------------------ incoherence processing (Hadamard + R pair)
+def _ip_case(seed=41, B=1, H=2, N=256, D=64):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, N, D))
+    k = rng.standard_normal((B, H, N, D)) + 2.0 * rng.standard_normal((B, H, 1, D))
+    q[..., 3] *= 30.0
+    k[..., 5] *= 10.0
+    q, k = (torch.from_numpy(a).to(torch.bfloat16) for a in (q, k))
+    signs = np.where(rng.random(D) < 0.5, -1, 1).astype(np.int8)
+    mu = orc.quantize(k, "k").k_mean
+    return q, k, signs, mu
+
+
+def test_incoherence_preserves_every_score():
+    """Q' K'^T = Q (K - mu)^T: H S is orthonormal and R^-1 R = I (FP32
+    outputs, so within FP32 rounding)."""
+    q, k, signs, mu = _ip_case()
+    qo, ko, _ = orc.incoherence(q, k, signs, mu)
+    S = np.einsum("bhid,bhjd->bhij", q.double().numpy(), k.double().numpy() - mu.astype(np.float64)[:, :, None, :])
+    S2 = np.einsum("bhid,bhjd->bhij", qo.astype(np.float64), ko.astype(np.float64))
+    assert np.abs(S2 - S).max() <= 1e-6 * np.abs(S).max()
+
+
+def test_incoherence_rotation_is_a_signed_orthonormal_hadamard():
+    """Undoing R gives the rotated rows Q H S: each row keeps its norm, and a
+    one-hot row (channel c, value a) becomes a (-1)^popcount(c & j) s_j /
+    sqrt(D) in every column j (Sylvester Hadamard, QuIP#-style signs)."""
+    q, k, signs, mu = _ip_case()
+    D = q.shape[-1]
+    qo, ko, r = orc.incoherence(q, k, signs, mu)
+    qrot = qo.astype(np.float64) * r[:, :, None, :]
+    assert np.allclose(np.linalg.norm(qrot, axis=-1), np.linalg.norm(q.double().numpy(), axis=-1), rtol=1e-6)
+    c, a = 37, 3.0
+    one = torch.zeros((1, 1, 16, D), dtype=torch.bfloat16)
+    one[0, 0, :, c] = a
+    q1, _, r1 = orc.incoherence(one, torch.ones_like(one), signs)
+    row = q1[0, 0, 0].astype(np.float64) * r1[0, 0]
+    expect = np.array([a * (-1) ** bin(c & j).count("1") * signs[j] / math.sqrt(D) for j in range(D)])
+    assert np.allclose(row, expect, rtol=1e-6, atol=0)
+
+
+def test_incoherence_r_balances_channels_and_minimises_energy():
+    """Each channel of Q' and K' has the same RMS, and no other diagonal
+    scaling of the rotated pair has a smaller total squared magnitude."""
+    q, k, signs, mu = _ip_case()
+    qo, ko, r = orc.incoherence(q, k, signs, mu)
+    Q, K = qo.astype(np.float64), ko.astype(np.float64)
+    rq, rk = np.sqrt((Q ** 2).mean(2)), np.sqrt((K ** 2).mean(2))
+    assert np.abs(rq / rk - 1).max() <= 1e-5
+    e0 = (Q ** 2).sum() + (K ** 2).sum()
+    rng = np.random.default_rng(42)
+    for _ in range(20):
+        w = np.exp(0.1 * rng.standard_normal(r.shape))[:, :, None, :]  # another diagonal R
+        assert (Q ** 2 / w ** 2).sum() + (K ** 2 * w ** 2).sum() >= e0 * (1 - 1e-9)
+
+
+def test_f32_row_quantiser_equals_the_bf16_quantiser():
+    """On bf16-representable rows the FP32-input quantiser writes the same
+    bytes and tensor scale as the bf16 quantiser (Q layout, no smoothing)."""
+    q, k, _ = wl.prefill_inputs("tiny")
+    for x, ss in ((q, False), (k, True)):
+        a = orc.quantize(x, "q", smooth=False, search=ss)
+        b = orc.quantize_rows_f32(x.float().numpy(), search=ss)
+        assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales, b.scales) and a.g == b.g
+        assert np.array_equal(a.ss_off, b.ss_off)
+
+
 # ------------------------------------------------ sink-aware mixed-precision decode
 def _exact_decode(q, k, v, sm):
     """Exact FP64 decode on raw operands: q [B,Hq,D], k/v [B,Hkv,L,D]."""
