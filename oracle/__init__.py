@@ -63,6 +63,8 @@ def lib():
         L.orc_decode_sink_f64.restype = i
         L.orc_thrift_select.argtypes = [P, P, i, i, i, i, i, i, P, P, P]
         L.orc_thrift_select.restype = i
+        L.orc_thrift_select_ex.argtypes = [P, P, P, i, i, i, i, i, i, i, P, P, P]
+        L.orc_thrift_select_ex.restype = i
         L.orc_num_threads.restype = i
         L.orc_quant_block.argtypes = [P, i, i, i, P, P, P, P]
         L.orc_block_err.argtypes, L.orc_block_err.restype = [P, i], f
@@ -341,15 +343,19 @@ def decode(q_bf16, kq: Quantized, vq: Quantized, sm_scale: float | None = None, 
 
 
 # ---------------------------------------------------------------- selector
-def thrift_select(q_bf16, k_bf16, causal: bool, frac_bp: int = 500, want_scores: bool = False):
+def thrift_select(q_bf16, k_bf16, causal: bool, frac_bp: int = 500, want_scores: bool = False,
+                  per_row: bool = False, k_mean=None):
+    """Block selector.  Default: raw keys, one budget per (b, h).  per_row:
+    one budget per query tile; k_mean [B,H,D]: pool the smoothed keys."""
     qb, kb = bf16_bits(q_bf16), bf16_bits(k_bf16)
     B, H, N, D = qb.shape
     T = (N + 127) // 128
     mask = np.zeros((B, H, T, T), np.uint8)
     nsel = np.zeros((B, H), np.int32)
     scores = np.zeros((B, H, T, T), np.float32) if want_scores else None
-    rc = lib().orc_thrift_select(_p(qb), _p(kb), B, H, N, D, int(causal), int(frac_bp), _p(mask), _p(nsel),
-                                 _p(scores))
+    km = None if k_mean is None else np.ascontiguousarray(k_mean, dtype=np.float32)
+    rc = lib().orc_thrift_select_ex(_p(qb), _p(kb), _p(km), B, H, N, D, int(causal), int(frac_bp), int(per_row),
+                                    _p(mask), _p(nsel), _p(scores))
     if rc != 0:
         raise ValueError(f"orc_thrift_select failed: {rc}")
     return (mask, nsel, scores) if want_scores else (mask, nsel)

@@ -716,26 +716,39 @@ static int cmp_scored(const void* a, const void* b)
     return (x->idx > y->idx) - (x->idx < y->idx);
 }
 
-/* Mean of one 128-row tile of raw bf16 rows, per channel: FP32 sum over the
- * rows in ascending order, divided by the row count, rounded to bf16. */
-static void pool_tile(const uint16_t* x, int r0, int r1, int D, float* out)
+/* Mean of one 128-row tile of bf16 rows, per channel: FP32 sum over the
+ * rows in ascending order (of fl(x - mu_c) when mu is given, else of x),
+ * divided by the row count, rounded to bf16. */
+static void pool_tile(const uint16_t* x, const float* mu, int r0, int r1, int D, float* out)
 {
     for (int c = 0; c < D; c++) {
         float acc = 0.0f;
-        for (int r = r0; r < r1; r++) acc = acc + bf16_to_f32(x[(size_t)r * D + c]);
+        for (int r = r0; r < r1; r++) {
+            float v = bf16_to_f32(x[(size_t)r * D + c]);
+            if (mu) v = v - mu[c];
+            acc = acc + v;
+        }
         out[c] = bf16_to_f32(orc_f32_to_bf16(acc / (float)(r1 - r0)));
     }
 }
 
 /*
- * Select the top frac_bp/10000 of valid (query tile, key tile) blocks per
- * (batch, head) by the score qbar_t . kbar_u (FP32 fmaf chain over channels
- * ascending).  Valid blocks: all, or u <= t when causal.  The count is
- * ceil(n_valid * frac_bp / 10000).  mask: [B,H,T,T] (1 = high precision);
- * nsel (nullable): [B,H]; scores (nullable): [B,H,T,T].
+ * Select the top frac_bp/10000 of valid (query tile, key tile) blocks by the
+ * score qbar_t . kbar_u (FP32 fmaf chain over channels ascending).  Valid
+ * blocks: all, or u <= t when causal.  Ranking: score descending, then the
+ * lower block index.
+ *  per_row = 0: one budget per (batch, head), ceil(n_valid * frac_bp / 10000);
+ *  per_row = 1: one budget per query tile t, ceil(n_valid_t * frac_bp / 10000)
+ *               over that row's valid key tiles.
+ *  k_mean (nullable, [B,H,D]): pool the smoothed keys fl(k - mu) instead of
+ *               the raw ones.  The per-row ranking is unchanged by any channel
+ *               offset up to the bf16 rounding of the means, since the offset
+ *               shifts every score of a row by the same q_t . mu.
+ * mask: [B,H,T,T] (1 = high precision); nsel (nullable): [B,H] blocks
+ * selected; scores (nullable): [B,H,T,T].
  */
-int orc_thrift_select(const uint16_t* q, const uint16_t* k, int B, int H, int N, int D, int causal, int frac_bp,
-                      uint8_t* mask, int32_t* nsel, float* scores)
+int orc_thrift_select_ex(const uint16_t* q, const uint16_t* k, const float* k_mean, int B, int H, int N, int D,
+                         int causal, int frac_bp, int per_row, uint8_t* mask, int32_t* nsel, float* scores)
 {
     if (N <= 0 || D <= 0 || frac_bp < 0 || frac_bp > 10000) return -1;
     int T = (N + TILE - 1) / TILE;
@@ -744,17 +757,19 @@ int orc_thrift_select(const uint16_t* q, const uint16_t* k, int B, int H, int N,
     for (long bh = 0; bh < BH; bh++) {
         const uint16_t* qb = q + (size_t)bh * N * D;
         const uint16_t* kb = k + (size_t)bh * N * D;
+        const float* mu = k_mean ? k_mean + (size_t)bh * D : NULL;
         float* qbar = (float*)malloc(sizeof(float) * T * D);
         float* kbar = (float*)malloc(sizeof(float) * T * D);
         scored_t* list = (scored_t*)malloc(sizeof(scored_t) * (size_t)T * T);
         for (int t = 0; t < T; t++) {
             int r1 = (t + 1) * TILE < N ? (t + 1) * TILE : N;
-            pool_tile(qb, t * TILE, r1, D, qbar + (size_t)t * D);
-            pool_tile(kb, t * TILE, r1, D, kbar + (size_t)t * D);
+            pool_tile(qb, NULL, t * TILE, r1, D, qbar + (size_t)t * D);
+            pool_tile(kb, mu, t * TILE, r1, D, kbar + (size_t)t * D);
         }
-        long nvalid = 0;
         uint8_t* mb = mask + (size_t)bh * T * T;
+        long total = 0, nvalid = 0;
         for (int t = 0; t < T; t++) {
+            long row0 = nvalid;
             for (int u = 0; u < T; u++) {
                 float acc = 0.0f;
                 for (int c = 0; c < D; c++) acc = fmaf(qbar[(size_t)t * D + c], kbar[(size_t)u * D + c], acc);
@@ -765,16 +780,32 @@ int orc_thrift_select(const uint16_t* q, const uint16_t* k, int B, int H, int N,
                 list[nvalid].idx = t * T + u;
                 nvalid++;
             }
+            if (per_row) {
+                long n = nvalid - row0, ksel = (n * (long)frac_bp + 9999) / 10000;
+                qsort(list + row0, (size_t)n, sizeof(scored_t), cmp_scored);
+                for (long i = 0; i < ksel; i++) mb[list[row0 + i].idx] = 1;
+                total += ksel;
+            }
         }
-        long ksel = (nvalid * (long)frac_bp + 9999) / 10000;
-        qsort(list, (size_t)nvalid, sizeof(scored_t), cmp_scored);
-        for (long i = 0; i < ksel; i++) mb[list[i].idx] = 1;
-        if (nsel) nsel[bh] = (int32_t)ksel;
+        if (!per_row) {
+            long ksel = (nvalid * (long)frac_bp + 9999) / 10000;
+            qsort(list, (size_t)nvalid, sizeof(scored_t), cmp_scored);
+            for (long i = 0; i < ksel; i++) mb[list[i].idx] = 1;
+            total = ksel;
+        }
+        if (nsel) nsel[bh] = (int32_t)total;
         free(qbar);
         free(kbar);
         free(list);
     }
     return 0;
+}
+
+/* The selector of the benchmark configuration: raw keys, one budget per head. */
+int orc_thrift_select(const uint16_t* q, const uint16_t* k, int B, int H, int N, int D, int causal, int frac_bp,
+                      uint8_t* mask, int32_t* nsel, float* scores)
+{
+    return orc_thrift_select_ex(q, k, NULL, B, H, N, D, causal, frac_bp, 0, mask, nsel, scores);
 }
 
 int orc_num_threads(void)

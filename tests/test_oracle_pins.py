@@ -578,6 +578,61 @@ def test_f32_row_quantiser_equals_the_bf16_quantiser():
         assert np.array_equal(a.ss_off, b.ss_off)
 
 
+# ------------------------------------------------ selector variants: per-row budget, smoothed keys
+def test_selector_per_row_budget_is_each_rows_top_k():
+    """Per-row budget: query tile t keeps ceil(n_valid_t * frac / 10000) of
+    its valid key tiles, the highest scores first and the lower key tile on a
+    tie (brute force over the returned scores)."""
+    q, k, _ = wl.prefill_inputs("longctx", B=1, H=2, N=2048, D=64)
+    T = 16
+    for causal in (False, True):
+        for frac in (500, 2500, 10000, 0):
+            mask, nsel, scores = orc.thrift_select(q, k, causal, frac, want_scores=True, per_row=True)
+            total = 0
+            for h in range(2):
+                for t in range(T):
+                    us = list(range(t + 1)) if causal else list(range(T))
+                    kt = (len(us) * frac + 9999) // 10000
+                    order = sorted(us, key=lambda u: (-float(scores[0, h, t, u]), u))
+                    want = np.zeros(T, np.uint8)
+                    want[order[:kt]] = 1
+                    assert np.array_equal(mask[0, h, t], want), (causal, frac, h, t)
+                    total += kt
+            assert nsel.sum() == total
+
+
+def test_selector_smoothed_keys_pool_the_centred_tiles():
+    """With a K mean the key tiles are pooled from fl(k - mu): the scores are
+    the FP64 dot products of the bf16 means of the centred tiles."""
+    q, k, _ = wl.prefill_inputs("longctx", B=1, H=2, N=1024, D=64)
+    mu = orc.quantize(k, "k").k_mean
+    _, _, scores = orc.thrift_select(q, k, False, 500, want_scores=True, k_mean=mu)
+    T = 8
+    ks = (k.float().numpy() - mu[:, :, None, :]).astype(np.float32)
+    qm = torch.from_numpy(q.float().numpy().reshape(1, 2, T, 128, 64).sum(3) / 128).to(torch.bfloat16).double()
+    km = torch.from_numpy(ks.reshape(1, 2, T, 128, 64).sum(3) / 128).to(torch.bfloat16).double()
+    ref = torch.einsum("bhtc,bhuc->bhtu", qm, km).numpy()
+    assert np.allclose(scores, ref, rtol=1e-5, atol=1e-4 * np.abs(ref).max())
+
+
+def test_selector_per_row_ranking_ignores_a_channel_offset():
+    """A K channel offset mu shifts every score of query tile t by the same
+    q_t . mu, so a per-row budget picks (up to the bf16 rounding of the tile
+    means) the same blocks from raw and from smoothed keys, while a per-head
+    budget does not: on the LLM workload's N(0, 3^2) channel offsets the two
+    per-head masks barely overlap."""
+    q, k, _ = wl.prefill_inputs("llm", B=1, H=4, N=4096, D=128)
+    mu = orc.quantize(k, "k").k_mean
+
+    def jaccard(per_row):
+        a, _ = orc.thrift_select(q, k, True, 500, per_row=per_row)
+        b, _ = orc.thrift_select(q, k, True, 500, per_row=per_row, k_mean=mu)
+        return (a & b).sum() / (a | b).sum()
+
+    assert jaccard(True) >= 0.85
+    assert jaccard(False) <= 0.5
+
+
 # ------------------------------------------------ sink-aware mixed-precision decode
 def _exact_decode(q, k, v, sm):
     """Exact FP64 decode on raw operands: q [B,Hq,D], k/v [B,Hkv,L,D]."""
