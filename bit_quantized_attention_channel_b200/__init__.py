@@ -87,6 +87,59 @@ def _check(fn, code):
         raise SAError(fn, code)
 
 
+def _tensor(name, t, dtype, ndim, shape=None):
+    """Raise unless t is a contiguous CUDA tensor of dtype with ndim dims
+    (and the given shape)."""
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.dim() != ndim or (shape is not None and tuple(t.shape) != tuple(shape)):
+        want = tuple(shape) if shape is not None else f"{ndim} dims"
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {want}")
+
+
+def _bf16(name, t, ndim, shape=None):
+    import torch
+
+    _tensor(name, t, torch.bfloat16, ndim, shape)
+
+
+def _nvfp4(name, t, shape=None, v_layout=None):
+    """Raise unless t is an NVFP4Tensor of the shape (V layout or not)."""
+    if not isinstance(t, NVFP4Tensor):
+        raise TypeError(f"{name}: expected an NVFP4Tensor, got {type(t).__name__}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if v_layout is not None and (t.role == "v") != v_layout:
+        raise ValueError(f"{name}: role {t.role!r} has the wrong layout here")
+
+
+def _on_device(name, t):
+    """Raise unless an NVFP4Tensor's buffers are in device memory."""
+    for part in ("codes", "scales", "g"):
+        if not getattr(t, part).is_cuda:
+            raise ValueError(f"{name}.{part}: must be in device memory")
+
+
+def _mode(mode):
+    if mode not in SA_SCALE:
+        raise ValueError(f"mode {mode!r}: expected one of {sorted(SA_SCALE)}")
+    return SA_SCALE[mode]
+
+
+def _role(role):
+    if role not in SA_ROLE:
+        raise ValueError(f"role {role!r}: expected one of {sorted(SA_ROLE)}")
+    return SA_ROLE[role]
+
+
 def _empty(nbytes, device, dtype=None):
     import torch
 
@@ -116,10 +169,15 @@ def sa_quant_nvfp4(x, role: str, smooth: bool = True, mode: str = "max", f_lo: i
     """Quantise bf16 x [B,H,N,D] (CUDA) to NVFP4 (see include/sa.h)."""
     import torch
 
+    _bf16("x", x, 4)
     B, H, N, D = x.shape
-    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    r, m = _role(role), _mode(mode)
+    if out is not None:
+        _nvfp4("out", out, (B, H, N, D))
+        if out.role != role:
+            raise ValueError(f"out: role {out.role!r}, expected {role!r}")
+        _on_device("out", out)
     L = lib()
-    r = SA_ROLE[role]
     if out is None:
         codes = _empty(L.sa_codes_bytes(B, H, N, D, r), x.device)
         scales = _empty(L.sa_scales_bytes(B, H, N, D, r), x.device)
@@ -131,7 +189,7 @@ def sa_quant_nvfp4(x, role: str, smooth: bool = True, mode: str = "max", f_lo: i
     ws_bytes = L.sa_quant_workspace_size(B, H, N, D, r)
     ws = _empty(ws_bytes, x.device)
     _check("sa_quant_nvfp4",
-           L.sa_quant_nvfp4(_ptr(x), B, H, N, D, r, int(smooth), SA_SCALE[mode], f_lo, f_hi, _ptr(out.codes),
+           L.sa_quant_nvfp4(_ptr(x), B, H, N, D, r, int(smooth), m, f_lo, f_hi, _ptr(out.codes),
                             _ptr(out.scales), _ptr(out.g), _ptr(out.k_mean), _ptr(out.ss_off), _ptr(ws), ws_bytes,
                             _stream(stream)))
     return out
@@ -144,9 +202,21 @@ def sa_quant_nvfp4_qkv(q, k, v, smooth: bool = True, mode: str = "max", f_lo: in
     (NVFP4Tensor q, k, v); `out` may pass the three to reuse."""
     import torch
 
+    _bf16("q", q, 4)
     B, H, N, D = q.shape
-    for t in (q, k, v):
-        assert t.dtype == torch.bfloat16 and t.is_cuda and t.is_contiguous() and tuple(t.shape) == (B, H, N, D)
+    _bf16("k", k, 4, (B, H, N, D))
+    _bf16("v", v, 4, (B, H, N, D))
+    m = _mode(mode)
+    if out is not None:
+        if len(out) != 3:
+            raise ValueError("out: expected the (q, k, v) NVFP4Tensors of an earlier call")
+        for name, t, role in (("out[0]", out[0], "q"), ("out[1]", out[1], "k"), ("out[2]", out[2], "v")):
+            _nvfp4(name, t, (B, H, N, D))
+            if t.role != role:
+                raise ValueError(f"{name}: role {t.role!r}, expected {role!r}")
+            _on_device(name, t)
+        if smooth and out[1].k_mean is None:
+            raise ValueError("out[1]: smoothing needs a k_mean buffer")
     L = lib()
     if out is None:
         out = []
@@ -160,7 +230,7 @@ def sa_quant_nvfp4_qkv(q, k, v, smooth: bool = True, mode: str = "max", f_lo: in
     ws_bytes = L.sa_quant_qkv_workspace_size(B, H, N, D)
     ws = _empty(ws_bytes, q.device)
     _check("sa_quant_nvfp4_qkv",
-           L.sa_quant_nvfp4_qkv(_ptr(q), _ptr(k), _ptr(v), B, H, N, D, int(smooth), SA_SCALE[mode], f_lo, f_hi,
+           L.sa_quant_nvfp4_qkv(_ptr(q), _ptr(k), _ptr(v), B, H, N, D, int(smooth), m, f_lo, f_hi,
                                 _ptr(qt.codes), _ptr(qt.scales), _ptr(qt.g), _ptr(kt.codes), _ptr(kt.scales),
                                 _ptr(kt.g), _ptr(kt.k_mean), _ptr(vt.codes), _ptr(vt.scales), _ptr(vt.g), _ptr(ws),
                                 ws_bytes, _stream(stream)))
@@ -171,7 +241,9 @@ def sa_thrift_select(q, k, causal: bool, frac_bp: int = 500, stream=None):
     """(mask uint8 [B,H,T,T], nsel int32 [B,H]) on the device."""
     import torch
 
+    _bf16("q", q, 4)
     B, H, N, D = q.shape
+    _bf16("k", k, 4, (B, H, N, D))
     T = (N + 127) // 128
     L = lib()
     mask = torch.empty(B, H, T, T, dtype=torch.uint8, device=q.device)
@@ -188,7 +260,21 @@ def sa_attn_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, causal: bool, sm
     """FP32 attention output [B,H,N,D] (and lse [B,H,N] if asked)."""
     import torch
 
+    _nvfp4("q", q, v_layout=False)
     B, H, N, D = q.shape
+    _nvfp4("k", k, (B, H, N, D), v_layout=False)
+    _nvfp4("v", v, (B, H, N, D), v_layout=True)
+    if mask is not None:
+        T = (N + 127) // 128
+        _tensor("mask", mask, torch.uint8, 4, (B, H, T, T))
+        for name, t in (("q_bf16", q_bf16), ("k_bf16", k_bf16), ("v_bf16", v_bf16)):
+            if t is None:
+                raise ValueError(f"{name}: the bf16 blocks of a mask need the raw inputs")
+            _bf16(name, t, 4, (B, H, N, D))
+    if out is not None:
+        _tensor("out", out, torch.float32, 4, (B, H, N, D))
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _on_device(name, t)
     dev = q.codes.device
     if out is None:
         out = torch.empty(B, H, N, D, dtype=torch.float32, device=dev)
@@ -206,8 +292,17 @@ def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.
     """q bf16 [B,Hq,D]; caches quantised as [B,Hkv,L,D]; returns FP32 [B,Hq,D]."""
     import torch
 
+    _bf16("q", q, 3)
     B, Hq, D = q.shape
+    _nvfp4("k", k, v_layout=False)
     _, Hkv, Lk, _ = k.shape
+    if k.shape[0] != B or k.shape[3] != D:
+        raise ValueError(f"k: shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    _nvfp4("v", v, tuple(k.shape), v_layout=True)
+    if out is not None:
+        _tensor("out", out, torch.float32, 3, (B, Hq, D))
+    _on_device("k", k)
+    _on_device("v", v)
     L = lib()
     if out is None:
         out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)

@@ -125,3 +125,48 @@ def test_fused_prepass_rejects_bad_arguments(L):
     assert L.sa_quant_nvfp4_qkv(n, n, n, 1, 1, 256, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 1
     # empty call
     assert L.sa_quant_nvfp4_qkv(n, n, n, 0, 1, 256, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 0
+
+
+def test_binding_validates_arguments_before_any_launch():
+    """The Python binding rejects host tensors, wrong dtypes, shapes, roles,
+    modes and masks with ValueError/TypeError before it loads a stream or
+    calls the library, so no host pointer ever reaches a kernel."""
+    import torch
+
+    x = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        sa.sa_quant_nvfp4(x, "q")
+    with pytest.raises(ValueError, match="dtype"):
+        sa.sa_quant_nvfp4(x.float(), "q")
+    with pytest.raises(TypeError):
+        sa.sa_quant_nvfp4(x.numpy(), "q")
+    with pytest.raises(ValueError, match="CUDA"):
+        sa.sa_quant_nvfp4_qkv(x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        sa.sa_thrift_select(x, x, True)
+    with pytest.raises(ValueError, match="CUDA"):
+        sa.sa_attn_decode_kvfp4(x[0], None, None)
+    with pytest.raises(ValueError, match="mode"):
+        sa._mode("maximum")
+    with pytest.raises(ValueError, match="role"):
+        sa._role("o")
+    with pytest.raises(ValueError, match="CUDA"):
+        sa._bf16("k", x, 4, (1, 2, 128, 128))      # device before shape
+
+    def fake(role, shape=(1, 2, 128, 64)):
+        b = torch.zeros(16, dtype=torch.uint8)
+        return sa.NVFP4Tensor(b, b, torch.ones(2), role, shape)
+
+    q, k, v = fake("q"), fake("k"), fake("v")
+    with pytest.raises(ValueError, match="layout"):
+        sa.sa_attn_fwd(q, k, fake("q"), True)        # V must carry the V layout
+    with pytest.raises(ValueError, match="layout"):
+        sa.sa_attn_fwd(fake("v"), k, v, True)
+    with pytest.raises(ValueError, match="shape"):
+        sa.sa_attn_fwd(q, fake("k", (1, 2, 256, 64)), v, True)
+    with pytest.raises(TypeError):
+        sa.sa_attn_fwd(q, k, "v", True)
+    with pytest.raises(ValueError, match="device memory"):
+        sa.sa_attn_fwd(q, k, v, True)                # host buffers never reach the library
+    with pytest.raises(ValueError, match="mask"):
+        sa.sa_attn_fwd(q, k, v, True, mask=torch.zeros(1, 2, 2, 2, dtype=torch.int32))
