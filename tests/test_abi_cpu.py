@@ -170,3 +170,15 @@ def test_binding_validates_arguments_before_any_launch():
         sa.sa_attn_fwd(q, k, v, True)                # host buffers never reach the library
     with pytest.raises(ValueError, match="mask"):
         sa.sa_attn_fwd(q, k, v, True, mask=torch.zeros(1, 2, 2, 2, dtype=torch.int32))
+
+
+def test_empty_calls_are_valid_and_launch_nothing(L):
+    """B = 0 or H = 0 is a valid empty call for every entry point: SA_OK, with
+    null buffers and no CUDA work (this host has no GPU)."""
+    n = None
+    assert L.sa_quant_nvfp4(n, 0, 1, 128, 64, 0, 0, 0, -2, 6, n, n, n, n, n, n, 0, n) == 0
+    assert L.sa_quant_nvfp4_qkv(n, n, n, 0, 1, 256, 128, 1, 0, -2, 6, *([n] * 10), n, 0, n) == 0
+    assert L.sa_attn_fwd(*([n] * 9), 0, 1, 128, 64, 0, 0.0, *([n] * 8)) == 0
+    assert L.sa_attn_fwd(*([n] * 9), 1, 0, 128, 64, 1, 0.0, *([n] * 8)) == 0
+    assert L.sa_attn_decode_kvfp4(*([n] * 7), 0, 8, 2, 256, 128, 0.0, n, n, 0, n) == 0
+    assert L.sa_thrift_select(n, n, 0, 1, 256, 64, 1, 500, n, n, n, 0, n) == 0
