@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -18,29 +19,35 @@ namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// The driver's tensor-map encoder, resolved once (thread-safe static
+// initialisation); null when the driver does not provide it.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         cudaDriverEntryPointQueryResult q;
         void* ptr = nullptr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    }();
     return fn;
 }
 
-// Streaming multiprocessors of the current device (cached per device).
+// Streaming multiprocessors of the current device (cached per device; host
+// threads may race on the first query, which stores the same value).
 int sm_count()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-    if (dev < 64 && cache[dev] > 0) return cache[dev];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev < 64) cache[dev] = n;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
@@ -322,13 +329,16 @@ sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v
 #define SA_PQ(DD, SS, SM)                                                                                      \
     do {                                                                                                       \
         const int smem = (int)sizeof(PqSmem<DD>);                                                              \
-        static int per_sm = 0; /* set once, outside any stream capture */                                      \
+        /* set on the first call, outside any stream capture; racing first calls store the same value */     \
+        static std::atomic<int> per_sm_cache{0};                                                               \
+        int per_sm = per_sm_cache.load(std::memory_order_acquire);                                             \
         if (!per_sm) {                                                                                         \
             if (cudaFuncSetAttribute(prepass_quant_kernel<DD, SS, SM>,                                         \
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||      \
                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prepass_quant_kernel<DD, SS, SM>, 2 * DD, \
                                                               smem) != cudaSuccess || per_sm < 1)              \
                 return SA_ERR_CUDA;                                                                            \
+            per_sm_cache.store(per_sm, std::memory_order_release);                                             \
         }                                                                                                      \
         const unsigned gq = (unsigned)std::min<long>(3L * BH * T, (long)per_sm * sm_count());                  \
         prepass_quant_kernel<DD, SS, SM><<<gq, 2 * DD, smem, stream>>>(p);                                     \
@@ -439,24 +449,24 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
         const int smem = MX ? (int)(((sizeof(AttnSmem<DD>) + 1023) & ~(size_t)1023) + sizeof(MixedSmem<DD>) + \
                                     1024)                                                                   \
                             : 116 * 1024; /* one CTA per SM: the CTA owns all 512 TMEM columns */          \
-        static int attr_done = 0; /* attribute set once, outside any stream capture */                    \
-        if (!attr_done) {                                                                                   \
+        static std::atomic<int> attr_done{0}; /* set once, outside any stream capture */                \
+        if (!attr_done.load(std::memory_order_acquire)) {                                                   \
             if (cudaFuncSetAttribute(attn_fwd_kernel<DD, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
                                      smem) != cudaSuccess)                                                  \
                 return SA_ERR_CUDA;                                                                         \
-            attr_done = 1;                                                                                  \
+            attr_done.store(1, std::memory_order_release);                                                  \
         }                                                                                                   \
         attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
     } while (0)
 #define SA_ATTN_PP_LAUNCH(DD)                                                                               \
     do {                                                                                                    \
         const int smem = (int)sizeof(PpSmem<DD>) + 1024;                                                    \
-        static int attr_done = 0;                                                                           \
-        if (!attr_done) {                                                                                   \
+        static std::atomic<int> attr_done{0};                                                               \
+        if (!attr_done.load(std::memory_order_acquire)) {                                                   \
             if (cudaFuncSetAttribute(attn_fwd_pp_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                                      smem) != cudaSuccess)                                                  \
                 return SA_ERR_CUDA;                                                                         \
-            attr_done = 1;                                                                                  \
+            attr_done.store(1, std::memory_order_release);                                                  \
         }                                                                                                   \
         const long nitems = (long)B * H * ((p.T + 1) / 2);                                                \
         const int nsm = sm_count();                                                                         \
@@ -531,22 +541,22 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
     dim3 grid(nsplit, Hkv, B);
     if (D == 128) {
         const int smem = (int)sizeof(DecSmem<128>) + 1024;
-        static int attr_done = 0;
-        if (!attr_done) {
+        static std::atomic<int> attr_done{0};
+        if (!attr_done.load(std::memory_order_acquire)) {
             if (cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
                 cudaSuccess)
                 return SA_ERR_CUDA;
-            attr_done = 1;
+            attr_done.store(1, std::memory_order_release);
         }
         decode_kernel<128><<<grid, 128, smem, stream>>>(tk, tv, p);
     } else {
         const int smem = (int)sizeof(DecSmem<64>) + 1024;
-        static int attr_done = 0;
-        if (!attr_done) {
+        static std::atomic<int> attr_done{0};
+        if (!attr_done.load(std::memory_order_acquire)) {
             if (cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
                 cudaSuccess)
                 return SA_ERR_CUDA;
-            attr_done = 1;
+            attr_done.store(1, std::memory_order_release);
         }
         decode_kernel<64><<<grid, 128, smem, stream>>>(tk, tv, p);
     }

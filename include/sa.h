@@ -24,6 +24,11 @@
  *    launch failures return SA_ERR_CUDA.  Device-side conditions (non-finite
  *    input, a pipeline wait that gave up) are recorded in a library status
  *    word that sa_device_status() reads.
+ *  - Host threads may call the entry points concurrently (each call with its
+ *    own buffers, workspace and stream); the library's only process-wide
+ *    state is per-kernel attribute and per-device caches, set race-free on
+ *    first use.  sa_quant_nvfp4_noalloc is the exception: its calls share one
+ *    scratch per device and must not overlap.
  *  - bf16 tensors are dense row-major [B, H, N, D].
  *  - Sizes: D in {64, 128}; N >= 1 with N % 16 == 0 (16 = NVFP4 block).
  *    B = 0 or H = 0 is a valid empty call that launches nothing.
