@@ -10,6 +10,7 @@ Entry points keep the C names:
   sa_quant_nvfp4        smoothing + NVFP4 pre-pass (max-scaling or ScaleSearch)
   sa_quant_nvfp4_qkv    the same for Q, K and V of one shape in two launches
   sa_thrift_select      high-precision block selector
+  sa_thrift_select_ex   the selector with per-row budgets / smoothed-K pooling
   sa_attn_fwd           NVFP4 attention forward (optionally with bf16 blocks)
   sa_attn_decode_kvfp4  decode over an NVFP4 KV cache
 """
@@ -62,6 +63,8 @@ def lib():
         L.sa_select_workspace_size.argtypes, L.sa_select_workspace_size.restype = [I, I, I, I], Z
         L.sa_thrift_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P, Z, P]
         L.sa_thrift_select.restype = I
+        L.sa_thrift_select_ex.argtypes = [P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        L.sa_thrift_select_ex.restype = I
         L.sa_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, P, P, P, P, P, P]
         L.sa_attn_fwd.restype = I
         L.sa_decode_workspace_size.argtypes, L.sa_decode_workspace_size.restype = [I, I, I, I, I], Z
@@ -252,6 +255,30 @@ def sa_thrift_select(q, k, causal: bool, frac_bp: int = 500, stream=None):
     ws = _empty(ws_bytes, q.device)
     _check("sa_thrift_select", L.sa_thrift_select(_ptr(q), _ptr(k), B, H, N, D, int(causal), int(frac_bp), _ptr(mask),
                                                   _ptr(nsel), _ptr(ws), ws_bytes, _stream(stream)))
+    return mask, nsel
+
+
+def sa_thrift_select_ex(q, k, causal: bool, frac_bp: int = 500, per_row: bool = False, k_mean=None,
+                        stream=None):
+    """sa_thrift_select with a per-query-tile budget (per_row) and/or keys
+    pooled after subtracting k_mean (float32 [B,H,D], device).  Returns
+    (mask uint8 [B,H,T,T], nsel int32 [B,H]) on the device."""
+    import torch
+
+    _bf16("q", q, 4)
+    B, H, N, D = q.shape
+    _bf16("k", k, 4, (B, H, N, D))
+    if k_mean is not None:
+        _tensor("k_mean", k_mean, torch.float32, 3, (B, H, D))
+    T = (N + 127) // 128
+    L = lib()
+    mask = torch.empty(B, H, T, T, dtype=torch.uint8, device=q.device)
+    nsel = torch.empty(B, H, dtype=torch.int32, device=q.device)
+    ws_bytes = L.sa_select_workspace_size(B, H, N, D)
+    ws = _empty(ws_bytes, q.device)
+    _check("sa_thrift_select_ex",
+           L.sa_thrift_select_ex(_ptr(q), _ptr(k), _ptr(k_mean), B, H, N, D, int(causal), int(frac_bp),
+                                 int(per_row), _ptr(mask), _ptr(nsel), _ptr(ws), ws_bytes, _stream(stream)))
     return mask, nsel
 
 

@@ -12,7 +12,9 @@
 //   per head (column): running max over keys (shuffles + shared memory),
 //   P~ = exp2(S c - m), per 16 keys (16 lanes) scale E4M3(max p/6), E2M1 codes
 //   -> P^T (B operand: 8 rows x 128 keys, 64-byte swizzle) + scale atom
-//   O^T[D, 8] += V^T_tile (A) x P^T,  L[128, 8] += ones(A) x P^T
+//   O^T[D, 8] += V^T_tile (A) x P^T; the row sums l add up the dequantised
+//   P (code x scale) of each head on the CUDA cores (warp shuffles, then the
+//   four warps in a fixed order), rescaled with the same running max as O.
 // q is quantised in the kernel with the tensor-wide g from a preceding amax
 // pass (same block rule as the pre-pass: 16 channels, max-scaling).
 // Each split writes (m, l, O) unnormalised; decode_combine_kernel merges the
@@ -24,6 +26,20 @@
 
 namespace sa {
 
+// E2M1 code (low nibble) of one float: one conversion, round to nearest
+// even, saturating, sign kept.
+SA_DEV uint32_t e2m1_code1(float y)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0;\n\t.reg .b16 h;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n\t"
+        "mov.b16 h, {b0, b0};\n\t"
+        "cvt.u32.u16 %0, h;\n\t}"
+        : "=r"(out)
+        : "f"(0.0f), "f"(y));
+    return out & 15u;
+}
+
 constexpr int kSplit = 4096;
 constexpr int kDecN = 8;  // MMA N (query heads of a group, zero-padded)
 
@@ -31,15 +47,16 @@ template <int D>
 struct DecSmem {
     alignas(1024) uint8_t k[128 * D / 2];    // K tile (A), D/2-byte swizzle
     alignas(1024) uint8_t v[128 * 64];       // V^T tile (A): 128 rows (rows >= D stay zero), 64-byte swizzle
-    alignas(1024) uint8_t ones[128 * 64];    // constant A operand: E2M1 1.0
     alignas(1024) uint8_t q[kDecN * D / 2];  // q^T (B): 8 rows, D/2-byte swizzle
     alignas(1024) uint8_t p[kDecN * 64];     // P^T (B): 8 rows x 128 keys, 64-byte swizzle
     uint8_t ksf[D / 64 * 512];
     uint8_t vsf[2 * 512];
     alignas(16) uint8_t qsf[D / 64 * 512];
     uint8_t psf[2 * 512];
-    uint8_t onesf[512];
-    float rcp[128];  // reciprocals of the E4M3 scale values
+    float rcp[128];    // reciprocals of the E4M3 scale values
+    float lg2sc[128];  // log2 of each nonzero E4M3 scale value
+    float lred[4][kDecN];  // per-warp partial sums of the dequantised P
+    float lrun[kDecN];     // running l per column (query head)
     float red[4][kDecN];
     float mnew[kDecN];
     float alpha[kDecN];
@@ -49,7 +66,7 @@ struct DecSmem {
 };
 
 // TMEM columns (64 allocated)
-constexpr uint32_t DM_S = 0, DM_O = 8, DM_L = 16, DM_SFK = 24, DM_SFQ = 32, DM_SFV = 40, DM_SFP = 48, DM_SF1 = 56;
+constexpr uint32_t DM_S = 0, DM_O = 8, DM_SFK = 24, DM_SFQ = 32, DM_SFV = 40, DM_SFP = 48;
 
 struct DecParams {
     const uint16_t* q;  // bf16 [B, Hq, D]
@@ -111,12 +128,12 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     if (tid == 0) {
         tc_fence_after();
         for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
-        tc_cp_sf(tbase + DM_SF1, smem_u32(s.onesf));
     }
 
     float m2[kDecN];
 #pragma unroll
     for (int h = 0; h < kDecN; h++) m2[h] = -INFINITY;
+    if (tid < kDecN) s.mnew[tid] = -INFINITY;  // read after the first tile's barriers
     const int key0 = split * kSplit;
     const int nkeys = min(kSplit, p.L - key0);
     const int ntiles = nkeys / 128;
@@ -169,7 +186,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         __syncthreads();
         if (tid < kDecN) {
             const float tmax = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
-            const float mo = m2[tid];
+            const float mo = s.mnew[tid];  // the running max (-inf before the first tile)
             const float mn = fmaxf(mo, tmax * cexp);
             s.mnew[tid] = mn;
             s.alpha[tid] = ex2f(mo - mn);
@@ -189,8 +206,13 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
 #pragma unroll
             for (int o = 8; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
             const uint32_t sc = f32_to_e4m3(ex2f(bm) * (1.0f / 6.0f));
-            const float y = sc ? ex2f(x - lg2f(e4m3_to_f32(sc))) : 0.0f;
-            const uint32_t code = pack8_e2m1(y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 15u;
+            const float y = sc ? ex2f(x - s.lg2sc[sc]) : 0.0f;
+            const uint32_t code = e2m1_code1(y);
+            // this key's dequantised P (in units of 1/2688), summed over the tile's keys
+            float pv = e2m1_to_f32(code) * e4m3_to_f32(sc);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pv += __shfl_xor_sync(0xffffffffu, pv, o);
+            if (lane == 0) s.lred[warp][h] = pv;
             const uint32_t hi_code = __shfl_down_sync(0xffffffffu, code, 1);
             if ((lane & 1) == 0) {
                 const int byte = tid >> 1;        // key pair index within the 128 keys
@@ -231,6 +253,10 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (tid < kDecN) {  // l = alpha l + sum of this tile's dequantised P (warps in order)
+            const float t = (s.lred[0][tid] + s.lred[1][tid]) + (s.lred[2][tid] + s.lred[3][tid]);
+            s.lrun[tid] = (u > 0 ? s.lrun[tid] * s.alpha[tid] : 0.0f) + t;
+        }
         if (tid == 0) {
             tc_fence_after();
             for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
@@ -239,8 +265,6 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
                 const uint32_t acc = (u > 0 || kb > 0) ? 1u : 0u;
                 mma_fp4(tbase + DM_O, make_sdesc(smem_u32(s.v) + 32 * kb, 512, 16, 4), pd, idesc_fp4(128, kDecN),
                         tbase + DM_SFV + 4 * kb, tbase + DM_SFP + 4 * kb, acc);
-                mma_fp4(tbase + DM_L, make_sdesc(smem_u32(s.ones) + 32 * kb, 512, 16, 4), pd,
-                        idesc_fp4(128, kDecN), tbase + DM_SF1, tbase + DM_SFP + 4 * kb, acc);
             }
             tc_commit(&s.mma_bar);
         }
@@ -250,20 +274,20 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     }
 
     // ---- write this split's unnormalised O (lane = channel), l and m
-    uint32_t o[kDecN], l[kDecN];
+    uint32_t o[kDecN];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%16];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%17];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]),
-          "=r"(l[0]), "=r"(l[1]), "=r"(l[2]), "=r"(l[3]), "=r"(l[4]), "=r"(l[5]), "=r"(l[6]), "=r"(l[7])
-        : "r"(tbase + lane_off + DM_O), "r"(tbase + lane_off + DM_L)
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7])
+        : "r"(tbase + lane_off + DM_O)
         : "memory");
-    for (int h = 0; h < p.G; h++) {
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) {  // constant indices keep o and m2 in registers
+        if (h >= p.G) break;
         float* dst = p.part + (((size_t)b * p.Hq + hk * p.G + h) * p.nsplit + split) * (D + 2);
         if (tid < D) dst[tid] = __uint_as_float(o[h]);
         if (tid == 0) {
-            dst[D] = __uint_as_float(l[h]);
+            dst[D] = s.lrun[h];
             dst[D + 1] = m2[h];
         }
     }
@@ -290,8 +314,11 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    for (int i = tid; i < 128 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.ones)[i] = 0x22222222u;
-    for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
+    if (tid < 128) {  // (e - 7) + log2(1 + m/8) for normal bytes, -7 + log2(m/4) for subnormal ones
+        const uint32_t e = (uint32_t)tid >> 3, m = (uint32_t)tid & 7u;
+        const float sig = e ? log2f(1.0f + m * 0.125f) : log2f(m * 0.25f);
+        s.lg2sc[tid] = (e ? (float)((int)e - 7) : -7.0f) + sig;
+    }
     for (int i = tid; i < kDecN * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.p)[i] = 0u;
     for (int i = tid; i < 2 * 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.psf)[i] = 0u;
     for (int i = D * 64 / 4 + tid; i < 128 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.v)[i] = 0u;

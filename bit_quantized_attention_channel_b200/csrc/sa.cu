@@ -361,9 +361,9 @@ size_t sa_select_workspace_size(int B, int H, int N, int D)
     return select_ws_bytes(B, H, N, D);
 }
 
-sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, int N, int D, int causal,
-                           int frac_bp, uint8_t* mask_dev, int32_t* nsel_dev, void* ws_dev, size_t ws_bytes,
-                           cudaStream_t stream)
+sa_status sa_thrift_select_ex(const void* q_dev, const void* k_dev, const float* k_mean_dev, int B, int H, int N,
+                              int D, int causal, int frac_bp, int per_row, uint8_t* mask_dev, int32_t* nsel_dev,
+                              void* ws_dev, size_t ws_bytes, cudaStream_t stream)
 {
     if (B < 0 || H < 0 || N < 0 || frac_bp < 0 || frac_bp > 10000) return SA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
@@ -376,14 +376,29 @@ sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, i
     float* qbar = (float*)ws_dev;
     float* kbar = (float*)((char*)ws_dev + sa_align256(BH * T * D * sizeof(float)));
     float* scores = (float*)((char*)ws_dev + 2 * sa_align256(BH * T * D * sizeof(float)));
-    pool_kernel<<<dim3(T, (unsigned)BH, 2), 128, 0, stream>>>((const uint16_t*)q_dev, (const uint16_t*)k_dev, N, D, T,
-                                                             qbar, kbar);
+    pool_kernel<<<dim3(T, (unsigned)BH, 2), 128, 0, stream>>>((const uint16_t*)q_dev, (const uint16_t*)k_dev,
+                                                             k_mean_dev, N, D, T, qbar, kbar);
     SA_CHECK_LAUNCH();
     score_kernel<<<dim3(sa_cdiv(T, 32), sa_cdiv(T, 8), (unsigned)BH), 256, 0, stream>>>(qbar, kbar, D, T, scores);
     SA_CHECK_LAUNCH();
-    topk_kernel<<<(unsigned)BH, kTopkThreads, 0, stream>>>(scores, T, causal, frac_bp, mask_dev, nsel_dev);
+    if (per_row) {
+        if (nsel_dev && cudaMemsetAsync(nsel_dev, 0, BH * sizeof(int32_t), stream) != cudaSuccess) return SA_ERR_CUDA;
+        const size_t rows = BH * (size_t)T;
+        topk_row_kernel<<<(unsigned)((rows + kRowWarps - 1) / kRowWarps), 32 * kRowWarps, 0, stream>>>(
+            scores, (int)BH, T, causal, frac_bp, mask_dev, nsel_dev);
+    } else {
+        topk_kernel<<<(unsigned)BH, kTopkThreads, 0, stream>>>(scores, T, causal, frac_bp, mask_dev, nsel_dev);
+    }
     SA_CHECK_LAUNCH();
     return SA_OK;
+}
+
+sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, int N, int D, int causal,
+                           int frac_bp, uint8_t* mask_dev, int32_t* nsel_dev, void* ws_dev, size_t ws_bytes,
+                           cudaStream_t stream)
+{
+    return sa_thrift_select_ex(q_dev, k_dev, nullptr, B, H, N, D, causal, frac_bp, 0, mask_dev, nsel_dev, ws_dev,
+                               ws_bytes, stream);
 }
 
 sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,

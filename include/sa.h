@@ -204,6 +204,24 @@ sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, i
                            cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * sa_thrift_select_ex -- sa_thrift_select with two further readings of the
+ * selector that "ThriftAttention" leaves open (the page fixes only the share
+ * of high-precision blocks and the joint softmax):
+ *  k_mean_dev   NULL: pool raw K (as sa_thrift_select).  Else float [B,H,D]
+ *               channel means (the K pre-pass output): each key row is pooled
+ *               as fl(k - mu_c), the smoothed keys the NVFP4 path quantises.
+ *  per_row      0: one budget per (b,h) over all valid blocks (as
+ *               sa_thrift_select).  1: one budget per query tile t,
+ *               ceil(n_valid_t*frac_bp/10000) of its valid key tiles (u <= t
+ *               when causal), by (score descending, u ascending); nsel_dev
+ *               (if not NULL) receives the per-(b,h) total.
+ * Other arguments, workspace and errors as sa_thrift_select.
+ * ------------------------------------------------------------------------ */
+sa_status sa_thrift_select_ex(const void* q_dev, const void* k_dev, const float* k_mean_dev, int B, int H, int N,
+                              int D, int causal, int frac_bp, int per_row, uint8_t* mask_dev, int32_t* nsel_dev,
+                              void* ws_dev, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * sa_attn_fwd -- NVFP4 attention forward (prefill).
  * "Search Your Block Floating Point Scales!", "ScaleSearchAttention /
  * 네이티브 NVFP4 실행": Q K^T and P V as block-scaled FP4 tensor-core MMAs

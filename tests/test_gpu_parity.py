@@ -194,6 +194,33 @@ def test_select_bit_exact_full_size():
     assert np.array_equal(mg.cpu().numpy(), mo)
 
 
+@pytest.mark.parametrize("per_row,smoothed,causal,frac", [(True, False, True, 500), (True, False, False, 500),
+                                                          (False, True, True, 500), (True, True, True, 1500),
+                                                          (True, False, True, 0), (True, True, False, 10000)])
+def test_select_ex_bit_exact(per_row, smoothed, causal, frac):
+    """Per-query-tile budgets and smoothed-K pooling: masks and counts equal
+    the oracle's bit for bit (ragged N, several heads)."""
+    q, k, _ = inputs("longctx", H=3, N=1024 + 256 + 64)
+    # each side pools with its own channel means (bit-identical, checked by the quant tests)
+    km_gpu = gpu_quant(k, "k").k_mean if smoothed else None
+    km_orc = orc.quantize(k, "k").k_mean if smoothed else None
+    mg, ng = sa.sa_thrift_select_ex(q.cuda(), k.cuda(), causal, frac, per_row=per_row, k_mean=km_gpu)
+    status_ok()
+    mo, no = orc.thrift_select(q, k, causal, frac, per_row=per_row, k_mean=km_orc)
+    assert np.array_equal(ng.cpu().numpy(), no)
+    assert np.array_equal(mg.cpu().numpy(), mo)
+
+
+def test_select_ex_per_row_full_size():
+    """Per-row budget on the full long-context workload (B1 H32 N65536)."""
+    q, k, _ = inputs("longctx")
+    mg, ng = sa.sa_thrift_select_ex(q.cuda(), k.cuda(), True, 500, per_row=True)
+    status_ok()
+    mo, no = orc.thrift_select(q, k, True, 500, per_row=True)
+    assert np.array_equal(ng.cpu().numpy(), no)
+    assert np.array_equal(mg.cpu().numpy(), mo)
+
+
 @pytest.mark.parametrize("shape,smooth,mode", [({"N": 4096, "D": 128, "B": 2, "H": 16}, True, "max"),
                                                ({"N": 416, "D": 64}, True, "search"),
                                                ({"N": 352, "D": 128}, False, "max"),
