@@ -1,16 +1,23 @@
 """Benchmark of the NVFP4 attention hot path on B200.
 
-A step is one pass of the path over one batch: the NVFP4 pre-pass of Q, K
-(smoothed) and V, then the FP4 attention forward.  Default workload: LLM
-prefill B2 H16 N4096 D128 causal, max-scaling (seeded synthetic inputs).
+A step is one pass of the path over one batch of seeded synthetic input: the
+NVFP4 pre-pass of Q, K (smoothed) and V (plus the bf16-block selector when the
+workload has one), then the attention forward (or, for decode, the split-KV
+decode over a cache quantised once before timing).
 Metric: FP4 attention TOPS = 4*B*H*N^2*D / t (causal halved), t = step time.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llm]
+The headline workload is the long-context mixed-precision prefill (B1 H32
+N65536 D128 causal, top 5% of blocks in bf16), the largest configuration that
+fits one GPU; the LLM prefill (max-scaling and ScaleSearch), the video-shaped
+prefill and the NVFP4-KV decode are measured in the same run and nested in the
+line under "workloads".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME [--only]]
                   [--mode max|search] [--impl ours|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica (the path has no
 cross-GPU exchange), timing is the max over ranks, value is the job total.
---impl reference times the CPU oracle on a bounded sample of the same workload.
+--impl reference times the CPU oracle on bounded samples of the same workload.
 """
 from __future__ import annotations
 
@@ -38,13 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch of the dominant kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum) on a batch slice of the same
-# workload, scaled by the units of the full launch (traffic grows with the
-# batch: each NVFP4 code and scale byte is read once).  Keyed by workload and
-# kernel; any other pair reports null.
-MEASURED_TRAFFIC = {
-    ("llm", "attn_fwd_pp_kernel<128>"): 14.74e6 * 2,  # B1 slice x 2
-    ("decode", "decode_kernel<128> + combine"): 305.7e6 * 4,  # B8 slice x 4
-}
+# workload, scaled by the units of the full launch.  Keyed by workload, scale
+# mode and kernel; any other key (or a kernel changed since its capture)
+# reports null.
+MEASURED_TRAFFIC = {}
 
 
 def peaks():
@@ -219,44 +223,79 @@ def hbm_bytes_decode(w):
     return kv + w.B * w.H * w.D * (2 + 4)
 
 
-def cpu_baseline(w, mode, budget_s=20.0):
-    """Oracle (plain C, OpenMP) on a bounded sample: full pre-pass of Q, K, V
-    plus attention for whole query tiles of every head, timed separately;
-    throughput = sampled FLOPs / (attention time + pre-pass time scaled to the
-    sampled share)."""
+def prepass_bytes(w):
+    """Algorithmic bytes of one pre-pass call: one bf16 read of Q, K and V
+    plus their NVFP4 codes and scales written (2 + 0.5 + 0.0625 B per element)."""
+    return 3 * w.B * w.H * w.N * w.D * 2.5625
+
+
+def attn_algorithmic_bytes(w):
+    """HBM bytes one attention launch must move: NVFP4 Q, K, V once (codes +
+    scales) and the FP32 output (plus, with bf16 blocks, nothing more is
+    counted: their raw tiles are re-reads of inputs already counted)."""
+    el = w.B * w.H * w.N * w.D
+    return 3 * el * 0.5625 + el * 4
+
+
+# ---------------------------------------------------------------- CPU oracle
+def cpu_sample_step(w, mode, q, k, v, tiles):
+    """One bounded sample of the hot path on the CPU oracle over the
+    single-head inputs (q, k, v): pre-pass of that head, the selector when the
+    workload has bf16 blocks, then FP64 attention of the given query tiles.
+    Returns (sampled FLOPs, seconds charged to them, wall seconds)."""
     import numpy as np
 
     import oracle as orc
 
-    q, k, v = wl.prefill_inputs(w)
     ss = mode == "search"
+    N, D = w.N, w.D
     t0 = time.perf_counter()
     qo, ko, vo = orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss), orc.quantize(v, "v", search=ss)
-    t_quant = time.perf_counter() - t0
-    B, H, N, D = w.B, w.H, w.N, w.D
-    T = (N + 127) // 128
-    qd, kd, vd = qo.dequant(), ko.dequant(), vo.dequant()
-    rows_done, flops, t_attn = [], 0.0, 0.0
-    order = [T - 1, 0, T // 2, T // 4, 3 * T // 4] + list(range(T))
-    seen = set()
-    for t in order:
-        if t in seen:
-            continue
-        seen.add(t)
-        rows = np.arange(t * 128, min(N, t * 128 + 128), dtype=np.int32)
-        t1 = time.perf_counter()
-        orc.attn_f64(qd, kd, vd, w.causal, 1 / math.sqrt(D), True, rows=rows)
-        t_attn += time.perf_counter() - t1
-        keys = (rows + 1).sum() if w.causal else len(rows) * N
-        flops += 4.0 * B * H * keys * D
-        rows_done.append(t)
-        if t_attn + t_quant > budget_s:
-            break
-    share = flops / w.flops()
-    t_total = t_attn + t_quant * share
-    return {"value": flops / t_total / 1e12, "unit": "TOPS", "cores": orc.num_threads(), "kind": "oracle",
-            "sample": f"pre-pass of full Q,K,V ({t_quant:.1f} s, scaled by {share:.4f}) + FP64 attention of "
-                      f"{len(rows_done)}/{T} query tiles of all {B * H} heads ({t_attn:.1f} s)"}
+    mask = None
+    if w.thrift_bp:
+        mask, _ = orc.thrift_select(q, k, w.causal, w.thrift_bp)
+    t_pre = time.perf_counter() - t0
+    rows = np.concatenate([np.arange(t * 128, min(N, t * 128 + 128), dtype=np.int32) for t in tiles])
+    t1 = time.perf_counter()
+    if mask is not None:
+        orc.attention(qo, ko, vo, w.causal, rows=rows, mask=mask, q_bf16=q, k_bf16=k, v_bf16=v)
+    else:
+        orc.attention(qo, ko, vo, w.causal, rows=rows)
+    t_attn = time.perf_counter() - t1
+    keys = float((rows + 1).sum()) if w.causal else float(len(rows)) * N
+    flops = 4.0 * keys * D
+    head_flops = w.flops() / (w.B * w.H)
+    return flops, t_attn + t_pre * flops / head_flops, t_pre + t_attn
+
+
+def cpu_sample_tiles(w, step, ntiles=8):
+    """Query tiles of sample `step`: ntiles spread over the head, rotating."""
+    T = (w.N + 127) // 128
+    return sorted({(step * 7 + i * max(1, T // ntiles)) % T for i in range(ntiles)})
+
+
+def cpu_baseline(w, mode, budget_s=20.0):
+    """Oracle (plain C, OpenMP) timed on bounded samples of the workload: each
+    sample is one head's pre-pass (plus selector) and FP64 attention of 8 of
+    its query tiles; throughput = sampled FLOPs / (attention time + the share
+    of the head's pre-pass those FLOPs account for)."""
+    import oracle as orc
+
+    if w.kind == "decode":
+        return None
+    q, k, v = wl.prefill_inputs(w, B=1, H=1)
+    flops = secs = 0.0
+    n = 0
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < budget_s or n == 0:
+        f, s, _ = cpu_sample_step(w, mode, q, k, v, cpu_sample_tiles(w, n))
+        flops += f
+        secs += s
+        n += 1
+    return {"value": flops / secs / 1e12, "unit": "TOPS", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{n} samples of one head (B1 H1 N{w.N} D{w.D}, same recipe): its pre-pass"
+                      f"{' and selector' if w.thrift_bp else ''} plus FP64 attention of 8 query tiles each; "
+                      f"pre-pass time charged in proportion to the sampled FLOPs"}
 
 
 def max_over_ranks(values, pg, device):
@@ -276,22 +315,41 @@ def whole_job_tops(world, flops_per_rank, ms_max):
 
 
 def run_reference(args, w, rank, world):
+    """The oracle as the reference arm: W untimed and K timed steps, each one
+    bounded sample of the workload on the host cores."""
     if rank != 0:
         return
-    cb = cpu_baseline(w, args.mode, budget_s=max(5.0, 60.0 / max(1, args.steps + args.warmup)))
-    line = {"metric": METRIC, "value": cb["value"], "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": w.flops() / (cb["value"] * 1e12) * 1e3, "higher_is_better": True,
+    import oracle as orc
+
+    if w.kind == "decode":
+        print(json.dumps({"impl": "reference", "unavailable": "the decode workload has no CPU sample step"}))
+        return
+    q, k, v = wl.prefill_inputs(w, B=1, H=1)
+    for i in range(args.warmup):
+        cpu_sample_step(w, args.mode, q, k, v, cpu_sample_tiles(w, i))
+    flops = charged = wall = 0.0
+    for i in range(args.steps):
+        f, s, wsec = cpu_sample_step(w, args.mode, q, k, v, cpu_sample_tiles(w, args.warmup + i))
+        flops += f
+        charged += s
+        wall += wsec
+    value = flops / charged / 1e12
+    cb = {"value": value, "unit": "TOPS", "cores": orc.num_threads(), "kind": "oracle",
+          "sample": f"each step: one head (B1 H1 N{w.N} D{w.D}) pre-pass{' + selector' if w.thrift_bp else ''} "
+                    f"and FP64 attention of 8 query tiles; pre-pass charged in proportion to the sampled FLOPs"}
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": config_of(w, args.mode), "cpu_baseline": cb,
-            "e2e": {"value": cb["value"], "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def traffic_of(w, kname, args):
     """Measured DRAM bytes per launch for the full workload, else None."""
-    if args.batch is not None or args.mode != "max":
+    if args.batch is not None:
         return None
-    return MEASURED_TRAFFIC.get((w.name, kname))
+    return MEASURED_TRAFFIC.get((w.name, args.mode if w.kind != "decode" else "max", kname))
 
 
 def config_of(w, mode):
@@ -305,51 +363,22 @@ def config_of(w, mode):
     return c
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llm")
-    ap.add_argument("--mode", default="max", choices=["max", "search"])
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=None,
-                    help="override the workload's batch (a smaller slice for ncu captures; not a bench line)")
-    args = ap.parse_args()
-    args.warmup = max(3, args.warmup)
+def kernel_name(w):
+    if w.kind == "decode":
+        return "decode_kernel<128> + combine"
+    return "attn_fwd_pp_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_pp_kernel<128>"
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = wl.WORKLOADS[args.workload]
-    if args.batch is not None:
-        import dataclasses
 
-        w = dataclasses.replace(w, B=args.batch, description=w.description + f" (batch {args.batch} slice)")
-
-    if args.impl == "reference":
-        run_reference(args, w, rank, world)
-        return
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
-
+def measure(w, mode, args, dev, pg, world, flush, want_e2e=True):
+    """Time one workload: W warm-up and K timed steps of the device-resident
+    path (L2 flushed between steps), then the same steps end to end from
+    pinned host memory.  Returns the fields of a bench line (rank 0 uses them)."""
     if w.kind == "decode":
         q, k, v = (t.to(dev) for t in wl.decode_inputs(w))
     else:
         q, k, v = (t.to(dev) for t in wl.prefill_inputs(w))
-    path = Path(w, args.mode, q, k, v)
+    path = Path(w, mode, q, k, v)
     path.capture()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -363,7 +392,7 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev.index) as clk:
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # evict L2 between steps (outside the step events)
@@ -380,16 +409,58 @@ def main():
     ms_attn = sum(a.elapsed_time(b) for a, b in aevs) / args.steps
     ms, ms_attn = max_over_ranks([ms, ms_attn], pg, dev)
 
-    # end to end through the C ABI from pinned host buffers, as a stream of
-    # steps: every step copies its inputs in, runs the path and copies its
-    # output back.  Two buffer sets and three streams let step i + 1's
-    # host->device copy overlap step i's compute and device->host copy
-    # (PCIe is full duplex); the L2 flush runs on the compute stream before
-    # each step.
+    e2e = None
+    if want_e2e:
+        e2e = measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v)
+
+    hbm, bf16, src = peaks()
+    fp4_peak = bf16 * 4.0  # dense FP4 = 4x dense bf16 (nominal ratio 9 / 2.25)
+    flops = flops_of(w)
+    kname = kernel_name(w)
+    if w.kind == "decode":
+        gbs = hbm_bytes_decode(w) / (ms_attn * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "peak_source": f"{src} copy bandwidth", "traffic": traffic_of(w, kname, args),
+                "traffic_unit": "DRAM bytes per launch (ncu, batch slice scaled)", "ms_per_launch": ms_attn,
+                "algorithmic_bytes": hbm_bytes_decode(w)}
+        value = whole_job_tops(world, flops, ms)
+    else:
+        achieved = flops / (ms_attn * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak,
+                "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
+                "traffic": traffic_of(w, kname, args),
+                "traffic_unit": "DRAM bytes per launch (ncu, batch slice scaled; the FP32 output's write-back "
+                                "that leaves L2 after the kernel ends is not in the kernel's count)",
+                "algorithmic_bytes": attn_algorithmic_bytes(w), "ms_per_launch": ms_attn}
+        value = whole_job_tops(world, flops, ms)
+    out = {"value": value, "ms_per_step": ms, "config": config_of(w, mode), "roofline": roof,
+           "gpu_launches": kernels_per_step(w) * args.steps, "clocks": clk.summary(), "wall_s": t_wall}
+    if w.kind != "decode":
+        ms_pre = ms - ms_attn  # the pre-pass (and selector) share of the step, between the graphs
+        pb = prepass_bytes(w)
+        out["prepass"] = {"ms": ms_pre, "algorithmic_bytes": pb, "achieved_gbs": pb / (ms_pre * 1e-3) / 1e9,
+                          "frac_of_hbm": pb / (ms_pre * 1e-3) / 1e9 / hbm,
+                          "note": "step time minus attention time (includes the selector when the workload has "
+                                  "bf16 blocks, and the L2 flush's write-backs)"}
+    if e2e is not None:
+        out["e2e"] = {"value": whole_job_tops(world, flops, e2e["ms"]), "unit": "TOPS",
+                      "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+    del path
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
+    """End to end through the C ABI from pinned host buffers, as a stream of
+    steps: every step copies its inputs in, runs the path and copies its
+    output back.  Two buffer sets and three streams let step i + 1's
+    host->device copy overlap step i's compute and device->host copy (PCIe
+    is full duplex); the L2 flush runs on the compute stream before each step."""
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     e2e_paths, houts = [], []
     for _ in range(2):
-        pth = Path(w, args.mode, torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        pth = Path(w, mode, torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
         pth.st.update({kk: path.st[kk] for kk in ("kc", "vc") if kk in path.st})
         e2e_paths.append(pth)
         houts.append(torch.empty(path.st["o"].shape, dtype=torch.float32).pin_memory())
@@ -439,44 +510,84 @@ def main():
     last = houts[(args.warmup + args.steps - 1) % 2]
     if not torch.equal(last, path.st["o"].cpu()):
         raise RuntimeError("end-to-end stream produced a different output than the resident path")
-    (e2e,) = max_over_ranks([e_start.elapsed_time(e_end) / args.steps], pg, dev)
-    h2d = inputs_of(e2e_paths[0])
-    hout = houts[0]
-    h2d_bytes = sum(src.numel() * src.element_size() for _, src in h2d)
+    (ms,) = max_over_ranks([e_start.elapsed_time(e_end) / args.steps], pg, dev)
+    h2d = sum(src.numel() * src.element_size() for _, src in inputs_of(e2e_paths[0]))
+    return {"ms": ms, "h2d": h2d, "d2h": houts[0].numel() * 4}
+
+
+# The workload BASELINE's metric is quoted on when nothing is named: the
+# largest configuration that fits one GPU (the long-context mixed prefill);
+# the others are measured in the same run and nested in the line.
+HEADLINE = ("longctx", "max")
+OTHERS = [("llm", "max"), ("llm", "search"), ("video", "search"), ("decode", "max")]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE[0])
+    ap.add_argument("--mode", default=None, choices=["max", "search"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only", action="store_true", help="measure the named workload alone (no nested workloads)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (a smaller slice for ncu captures; not a bench line)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.WORKLOADS[args.workload]
+    if args.mode is None:
+        args.mode = "search" if w.scale_modes == ("search",) else "max"
+    if args.batch is not None:
+        import dataclasses
+
+        w = dataclasses.replace(w, B=args.batch, description=w.description + f" (batch {args.batch} slice)")
+        args.only = True
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    head = measure(w, args.mode, args, dev, pg, world, flush, want_e2e=not args.no_e2e)
+    nested = []
+    if not args.only and args.workload == HEADLINE[0]:
+        for name, mode in OTHERS:
+            r = measure(wl.WORKLOADS[name], mode, args, dev, pg, world, flush, want_e2e=not args.no_e2e)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and wl.WORKLOADS[name].kind != "decode":
+                r["cpu_baseline"] = cpu_baseline(wl.WORKLOADS[name], mode, budget_s=6.0)
+            nested.append(r)
 
     if rank == 0:
-        hbm, bf16, src = peaks()
-        fp4_peak = bf16 * 4.0  # dense FP4 = 4x dense bf16 (nominal ratio 9 / 2.25)
-        flops = flops_of(w)
-        if w.kind == "decode":
-            gbs = hbm_bytes_decode(w) / (ms_attn * 1e-3) / 1e9
-            kname = "decode_kernel<128> + combine"
-            roof = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm,
-                    "unit": "GB/s", "frac": gbs / hbm, "peak_source": f"{src} copy bandwidth",
-                    "traffic": traffic_of(w, kname, args), "traffic_unit": "bytes per launch (ncu, batch slice scaled)",
-                    "ms_per_launch": ms_attn, "algorithmic_bytes": hbm_bytes_decode(w)}
-        else:
-            achieved = flops / (ms_attn * 1e-3) / 1e12
-            kname = "attn_fwd_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_pp_kernel<128>"
-            roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                    "frac": achieved / fp4_peak,
-                    "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
-                    "traffic": traffic_of(w, kname, args), "traffic_unit": "bytes per launch (ncu, batch slice scaled)",
-                    "ms_per_launch": ms_attn}
-        line = {
-            "metric": METRIC, "value": whole_job_tops(world, flops, ms), "unit": "TOPS", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
-            "config": config_of(w, args.mode),
-            "roofline": roof,
-            "e2e": {"value": whole_job_tops(world, flops, e2e), "unit": "TOPS",
-                    "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": hout.numel() * 4},
-            "gpu_launches": kernels_per_step(w) * args.steps,
-            "clocks": clk.summary(),
-            "wall_s": t_wall,
-        }
+        line = {"metric": METRIC, "value": head["value"], "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+                "config": head["config"], "roofline": head["roofline"]}
+        for key in ("prepass", "e2e", "gpu_launches", "clocks", "wall_s"):
+            if key in head:
+                line[key] = head[key]
+        line["gpu_launches"] = head["gpu_launches"] + sum(r["gpu_launches"] for r in nested)
         if world == 1 and not args.no_cpu_baseline and w.kind != "decode":
             line["cpu_baseline"] = cpu_baseline(w, args.mode)
+        if nested:
+            line["workloads"] = nested
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()

@@ -50,6 +50,7 @@ def lib():
         P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.sa_status_string.argtypes, L.sa_status_string.restype = [I], ctypes.c_char_p
         L.sa_device_status.argtypes, L.sa_device_status.restype = [P, I], I
+        L.sa_set_wait_cycles.argtypes, L.sa_set_wait_cycles.restype = [ctypes.c_longlong], None
         for n in ("sa_codes_bytes", "sa_scales_bytes"):
             getattr(L, n).argtypes, getattr(L, n).restype = [I, I, I, I, I], Z
         L.sa_quant_workspace_size.argtypes, L.sa_quant_workspace_size.restype = [I, I, I, I, I], Z
@@ -165,6 +166,12 @@ class NVFP4Tensor:
 def sa_device_status(reset: bool = True, stream=None) -> int:
     """Synchronise and return the library's device status word."""
     return lib().sa_device_status(_stream(stream), int(reset))
+
+
+def sa_set_wait_cycles(cycles: int = 0) -> None:
+    """Limit of every pipeline wait of the attention kernel in later calls,
+    in SM clock cycles (0: the default, about 2 s); see include/sa.h."""
+    lib().sa_set_wait_cycles(int(cycles))
 
 
 def sa_quant_nvfp4(x, role: str, smooth: bool = True, mode: str = "max", f_lo: int = -2, f_hi: int = 6,

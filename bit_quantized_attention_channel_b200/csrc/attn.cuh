@@ -1,33 +1,21 @@
-// attn.cuh -- NVFP4 attention forward on tcgen05 block-scaled MMAs.
+// attn.cuh -- parameters and constants shared by the NVFP4 attention kernels.
 //
 // "Search Your Block Floating Point Scales!" (gist.science summary),
 // "ScaleSearchAttention / 네이티브 NVFP4 실행": Q K^T and P V run natively in
 // NVFP4 on tensor cores with FP32 accumulation.  SageAttention3 article
-// (dasgeld.co): FP4 tensor-core attention on Blackwell.
+// (dasgeld.co): FP4 tensor-core attention on Blackwell.  "ThriftAttention:
+// 5%의 연산량으로 90%의 품질 유지": a few query-key blocks in high precision
+// inside one joint softmax.
 //
-// One CTA per (b, h, 128-query tile); thread i of the 128 owns query row i,
-// which is TMEM lane i of every accumulator.  Per key tile of 128:
-//   TMA K codes (128 x D/2 B, swizzled) + K scale atoms, V^T codes (D x 64 B)
-//   + V scale atoms -> tcgen05.cp scale atoms into TMEM ->
-//   S = Q K^T (kind::mxf4nvf4, M=128 N=128, D/64 MMAs of K=64) ->
-//   softmax rows from TMEM: running max m (log2 units), P~ = exp2(S c - m),
-//   per 16 keys: scale = E4M3(max p / 6) with p = 2688 P~, codes = E2M1(p/s)
-//   computed as exp2(S c + log2(2688) - m - log2 s) ->
-//   P codes to shared memory (64-byte swizzle, the MMA A layout), P scales to
-//   an atom -> rescale O and l in TMEM when the running max moved ->
-//   O += P V^T (N = D) and l += P 1 (N = 16, a constant all-ones operand), so
-//   l sums the dequantised P exactly on the tensor core.
-// Epilogue: out = O / l * g_V (FP32), lse = m ln2 + ln(l / 2688).
-//
-// MIXED variant ("ThriftAttention: 5%의 연산량으로 90%의 품질 유지": a few
-// query-key blocks in high precision, one joint softmax): where the block mask
-// is set, the key tile is instead loaded as raw bf16 K and V (TMA, 128-byte
-// swizzle), S = q.k - c_i with c_i = q_i.mean(K) comes from kind::f16 MMAs on
-// the raw bf16 Q tile (so FP4 and bf16 scores share one per-row offset), P is
-// rounded to bf16 and O_b += P V runs with V as an MN-major operand.  O_b is a
-// second TMEM accumulator (raw V units) and l_b a register; both are rescaled
-// with the same running max, and the epilogue merges
-// out = (O g_V / 2688 + O_b) / (l / 2688 + l_b).
+// Score arithmetic common to the kernels (log2 units throughout):
+//   NVFP4 block:  t = S c2, c2 = g_Q g_K sm_scale log2(e), S the block-scaled
+//                 MMA result of the codes;
+//   bf16 block:   t = (q.k - c_i) sm_scale log2(e), q.k from the raw bf16
+//                 inputs, c_i = q_i . mean(K) (so both kinds of block carry
+//                 the same per-row offset as the smoothed keys);
+//   running max m, P~ = 2^(t - m); NVFP4 P: per 16 keys, scale
+//   E4M3(max(2688 P~) / 6) and E2M1 codes of 2688 P~ / scale, computed as
+//   2^(t + log2(2688) - m - log2(scale)).
 #pragma once
 
 #include "tc.cuh"
@@ -52,42 +40,11 @@ struct AttnParams {
     int CKv;  // 64-key chunks of the V scale atoms per (b,h)
     int causal;
     float sm_scale;
-    const uint8_t* mask;  // MIXED: [B,H,T,T] high-precision block flags
+    const uint8_t* mask;  // mixed: [B,H,T,T] high-precision block flags
     const uint16_t* q_bf16;
-    const float* k_mean;  // MIXED: channel means of K (nullptr: not smoothed)
+    const float* k_mean;  // mixed: channel means of K (nullptr: not smoothed)
+    long long wait_cycles;  // limit of every pipeline wait (SM clock cycles)
 };
-
-template <int D>
-struct AttnSmem {
-    alignas(1024) uint8_t q[128 * D / 2];   // Q tile, K-major, D/2-byte swizzle
-    alignas(1024) uint8_t k[128 * D / 2];   // K tile
-    alignas(1024) uint8_t v[D * 64];        // V^T tile: D rows x 128 keys, 64-byte swizzle
-    alignas(1024) uint8_t p[128 * 64];      // P tile: 128 rows x 128 keys, 64-byte swizzle
-    alignas(1024) uint8_t ones[16 * 64];    // constant operand: 16 rows of E2M1 1.0
-    alignas(16) uint8_t qsf[D / 64 * 512];
-    uint8_t ksf[D / 64 * 512];
-    uint8_t vsf[2 * 512];
-    uint8_t psf[2 * 512];
-    uint8_t onesf[512];
-    uint64_t tma_bar;
-    uint64_t mma_bar;
-    uint32_t tmem_slot;
-    uint32_t flag;
-};
-
-// Raw bf16 operands of the high-precision blocks: each region is 128 rows x
-// 128 bytes (64 bf16) with the 128-byte swizzle.
-template <int D>
-struct MixedSmem {
-    alignas(1024) uint8_t qb[D / 64][16384];  // Q tile, K-major (channels)
-    alignas(1024) uint8_t kb[D / 64][16384];  // K tile, K-major
-    alignas(1024) uint8_t vb[D / 64][16384];  // V tile: rows = keys, MN-major (channels)
-    alignas(1024) uint8_t pb[2][16384];       // P tile bf16, K-major (keys)
-};
-
-// TMEM columns (512 allocated)
-constexpr uint32_t TM_S = 0, TM_O = 128, TM_L = 256, TM_SFQ = 272, TM_SFK = 280, TM_SFP = 288, TM_SFV = 296,
-                   TM_SF1 = 304, TM_OB = 320;
 
 SA_DEV float tmem_ld1_sync(uint32_t taddr)
 {
@@ -99,363 +56,6 @@ SA_DEV float tmem_ld1_sync(uint32_t taddr)
         : "r"(taddr)
         : "memory");
     return __uint_as_float(r);
-}
-
-// Multiply this warp's lanes of `ncols` accumulator columns by alpha.
-SA_DEV void tmem_scale_cols(uint32_t taddr, int ncols, float alpha)
-{
-    for (int c = 0; c < ncols; c += 32) {
-        float o[32];
-        tmem_ld32(taddr + c, o);
-        tmem_wait_ld();
-        reg_fence(o);
-#pragma unroll
-        for (int i = 0; i < 32; i++) o[i] *= alpha;
-        tmem_st32(taddr + c, o);
-    }
-    tmem_wait_st();
-}
-
-template <int D, bool MIXED>
-SA_DEV bool attn_body(AttnSmem<D>& s, MixedSmem<D>* mx, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
-                      const CUtensorMap* tm_v, const CUtensorMap* tm_qb, const CUtensorMap* tm_kb,
-                      const CUtensorMap* tm_vb, const AttnParams& p, int t, int bh, uint32_t tbase)
-{
-    constexpr int KB = D / 64;             // K=64 MMA steps for Q K^T
-    constexpr uint32_t QSW = D == 128 ? 4u : 6u;  // 64B / 32B swizzle
-    constexpr uint32_t QSBO = 8 * D / 2;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int row = t * 128 + tid;
-    const float c2 = p.q_g[0] * p.k_g[0] * p.sm_scale * kLog2e;
-    uint32_t tma_phase = 0, mma_phase = 0;
-
-    const int Tk = (p.N + 127) / 128;
-    const int nt = p.causal ? min(t + 1, Tk) : Tk;
-    const uint8_t* mrow = MIXED ? p.mask + ((size_t)bh * p.T + t) * p.T : nullptr;
-    bool row_mixed = false;
-    if (MIXED) {
-        if (tid == 0) {
-            uint32_t any = 0;
-            for (int u = 0; u < nt; u++) any |= mrow[u];
-            s.flag = any;
-        }
-        __syncthreads();
-        row_mixed = s.flag != 0;
-    }
-    if (tid == 0) {
-        mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + (row_mixed ? 128 * D * 2 : 0));
-        tma_load_3d(s.q, tm_q, &s.tma_bar, 0, t * 128, bh);
-        bulk_load(s.qsf, p.q_sf + ((size_t)bh * p.T + t) * KB * 512, KB * 512, &s.tma_bar);
-        if (MIXED && row_mixed)
-            for (int r = 0; r < D / 64; r++) tma_load_3d(mx->qb[r], tm_qb, &s.tma_bar, 64 * r, t * 128, bh);
-    }
-    // per-row offset of the high-precision scores: c_i = q_i . mean(K)
-    float crow = 0.0f;
-    if (MIXED && row_mixed && p.k_mean) {
-        const uint16_t* qr = p.q_bf16 + ((size_t)bh * p.N + min(row, p.N - 1)) * D;
-        const float* mu = p.k_mean + (size_t)bh * D;
-        for (int c = 0; c < D; c++) crow = __fmaf_rn(bf16_bits_to_f32(qr[c]), mu[c], crow);
-    }
-    const float cb = p.sm_scale * kLog2e;  // bf16 scores -> log2 units
-    if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
-    tma_phase ^= 1;
-    if (tid == 0) {
-        tc_fence_after();
-        for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + TM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
-        tc_cp_sf(tbase + TM_SF1, smem_u32(s.onesf));
-    }
-
-    float m2 = -INFINITY;
-    float lb = 0.0f;        // MIXED: sum of bf16 P over high-precision blocks
-    bool has_f = false, has_b = false;
-    for (int u = 0; u < nt; u++) {
-        const int nk = min(128, p.N - u * 128);
-        const int kblocks = nk > 64 ? 2 : 1;
-        if (MIXED && mrow[u]) {
-            // ================= high-precision (bf16) block =================
-            if (tid == 0) {
-                mbar_expect_tx(&s.tma_bar, 2 * 128 * D * 2);
-                for (int r = 0; r < D / 64; r++) {
-                    tma_load_3d(mx->kb[r], tm_kb, &s.tma_bar, 64 * r, u * 128, bh);
-                    tma_load_3d(mx->vb[r], tm_vb, &s.tma_bar, 64 * r, u * 128, bh);
-                }
-            }
-            if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
-            tma_phase ^= 1;
-            if (tid == 0) {
-                tc_fence_after();
-                for (int ks = 0; ks < D / 16; ks++)
-                    mma_bf16(tbase + TM_S, make_sdesc(smem_u32(mx->qb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                             make_sdesc(smem_u32(mx->kb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                             idesc_bf16(128, 128, 0), ks > 0);
-                tc_commit(&s.mma_bar);
-            }
-            if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
-            mma_phase ^= 1;
-            tc_fence_after();
-            float sv[128];
-#pragma unroll
-            for (int c = 0; c < 4; c++)
-                tmem_ld32(tbase + lane_off + TM_S + 32 * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
-            tmem_wait_ld();
-            reg_fence(sv);
-            const int kbase = u * 128;
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int jj = 0; jj < 128; jj++) {
-                const int j = kbase + jj;
-                const bool valid = j < p.N && (!p.causal || j <= row);
-                const float x = valid ? __fsub_rn(sv[jj], crow) * cb : -INFINITY;
-                sv[jj] = x;
-                tmax = fmaxf(tmax, x);
-            }
-            const float m2_new = fmaxf(m2, tmax);
-            const float msub = m2_new == -INFINITY ? 0.0f : m2_new;
-            const float alpha = ex2f(m2 - msub);
-            m2 = m2_new;
-            lb *= alpha;
-            // P in bf16 (A operand: 2 regions of 64 keys, 128-byte swizzle)
-#pragma unroll
-            for (int c = 0; c < 16; c++) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const __nv_bfloat162 pr = __floats2bfloat162_rn(ex2f(sv[8 * c + 2 * e] - msub),
-                                                                    ex2f(sv[8 * c + 2 * e + 1] - msub));
-                    lb += __low2float(pr);
-                    lb += __high2float(pr);
-                    w[e] = *reinterpret_cast<const uint32_t*>(&pr);
-                }
-                const int cc = c & 7;
-                *reinterpret_cast<uint4*>(mx->pb[c >> 3] + (tid >> 3) * 1024 + (tid & 7) * 128 +
-                                          ((cc ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                if (has_f) {
-                    tmem_scale_cols(tbase + lane_off + TM_O, D, alpha);
-                    const float l = tmem_ld1_sync(tbase + lane_off + TM_L);
-                    tmem_st1(tbase + lane_off + TM_L, l * alpha);
-                    tmem_wait_st();
-                }
-                if (has_b) tmem_scale_cols(tbase + lane_off + TM_OB, D, alpha);
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                for (int ks = 0; ks < 8; ks++)
-                    mma_bf16(tbase + TM_OB, make_sdesc(smem_u32(mx->pb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                             make_sdesc(smem_u32(mx->vb[0]) + 2048 * ks, 1024, 16384, 2), idesc_bf16(128, D, 1),
-                             (has_b || ks > 0) ? 1u : 0u);
-                tc_commit(&s.mma_bar);
-            }
-            if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
-            mma_phase ^= 1;
-            tc_fence_after();
-            has_b = true;
-            continue;
-        }
-        // ================= NVFP4 block =================
-        if (tid == 0) {
-            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
-            tma_load_3d(s.k, tm_k, &s.tma_bar, 0, u * 128, bh);
-            bulk_load(s.ksf, p.k_sf + ((size_t)bh * p.T + u) * KB * 512, KB * 512, &s.tma_bar);
-            tma_load_3d(s.v, tm_v, &s.tma_bar, 0, u * D, bh);
-            bulk_load(s.vsf, p.v_sf + ((size_t)bh * p.CKv + 2 * u) * 512, kblocks * 512, &s.tma_bar);
-        }
-        if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
-        tma_phase ^= 1;
-        if (tid == 0) {
-            tc_fence_after();
-            for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + TM_SFK + 4 * kb, smem_u32(s.ksf + 512 * kb));
-            for (int kb = 0; kb < kblocks; kb++) tc_cp_sf(tbase + TM_SFV + 4 * kb, smem_u32(s.vsf + 512 * kb));
-            for (int kb = 0; kb < KB; kb++)
-                mma_fp4(tbase + TM_S, make_sdesc(smem_u32(s.q) + 32 * kb, QSBO, 16, QSW),
-                        make_sdesc(smem_u32(s.k) + 32 * kb, QSBO, 16, QSW), idesc_fp4(128, 128),
-                        tbase + TM_SFQ + 4 * kb, tbase + TM_SFK + 4 * kb, kb > 0);
-            tc_commit(&s.mma_bar);
-        }
-        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- this row's 128 scores
-        float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; c++)
-            tmem_ld32(tbase + lane_off + TM_S + 32 * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
-        tmem_wait_ld();
-        reg_fence(sv);
-
-        const int kbase = u * 128;
-        float bmax[8];
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int blk = 0; blk < 8; blk++) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int j = kbase + blk * 16 + i;
-                const bool valid = j < p.N && (!p.causal || j <= row);
-                const float v = valid ? sv[blk * 16 + i] : -INFINITY;
-                sv[blk * 16 + i] = v;
-                mx = fmaxf(mx, v);
-            }
-            bmax[blk] = mx;
-            tmax = fmaxf(tmax, mx);
-        }
-        const float m2_new = fmaxf(m2, tmax * c2);
-        const float msub = m2_new == -INFINITY ? 0.0f : m2_new;
-        const float alpha = ex2f(m2 - msub);
-        uint32_t codes[16];
-        uint32_t scw0 = 0, scw1 = 0;
-#pragma unroll
-        for (int blk = 0; blk < 8; blk++) {
-            const float pmax = ex2f(fmaf(bmax[blk], c2, kLog2_2688 - msub));
-            const uint32_t sc = f32_to_e4m3(pmax * (1.0f / 6.0f));
-            const float bias = sc ? (kLog2_2688 - msub - lg2f(e4m3_to_f32(sc))) : -INFINITY;
-            float y[16];
-#pragma unroll
-            for (int i = 0; i < 16; i++) y[i] = ex2f(fmaf(sv[blk * 16 + i], c2, bias));
-            codes[2 * blk] = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-            codes[2 * blk + 1] = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-            if (blk < 4)
-                scw0 |= sc << (8 * blk);
-            else
-                scw1 |= sc << (8 * (blk - 4));
-        }
-        m2 = m2_new;
-
-        // ---- P codes (A operand, 64-byte swizzle) and scale atoms
-        uint8_t* prow = s.p + (tid >> 3) * 512 + (tid & 7) * 64;
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const int cs = c ^ ((tid & 7) >> 1);
-            *reinterpret_cast<uint4*>(prow + cs * 16) =
-                make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
-        }
-        *reinterpret_cast<uint32_t*>(s.psf + (tid & 31) * 16 + (tid >> 5) * 4) = scw0;
-        *reinterpret_cast<uint32_t*>(s.psf + 512 + (tid & 31) * 16 + (tid >> 5) * 4) = scw1;
-
-        // ---- rescale the accumulators when this warp's running max moved
-        if (MIXED) lb *= alpha;
-        if ((has_f || has_b) && __any_sync(0xffffffffu, alpha != 1.0f)) {
-            if (has_f) {
-                tmem_scale_cols(tbase + lane_off + TM_O, D, alpha);
-                const float l = tmem_ld1_sync(tbase + lane_off + TM_L);
-                tmem_st1(tbase + lane_off + TM_L, l * alpha);
-                tmem_wait_st();
-            }
-            if (MIXED && has_b) tmem_scale_cols(tbase + lane_off + TM_OB, D, alpha);
-        }
-
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            for (int kb = 0; kb < kblocks; kb++) tc_cp_sf(tbase + TM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
-            for (int kb = 0; kb < kblocks; kb++) {
-                const uint64_t pd = make_sdesc(smem_u32(s.p) + 32 * kb, 512, 16, 4);
-                const uint32_t acc = (has_f || kb > 0) ? 1u : 0u;
-                mma_fp4(tbase + TM_O, pd, make_sdesc(smem_u32(s.v) + 32 * kb, 512, 16, 4), idesc_fp4(128, D),
-                        tbase + TM_SFP + 4 * kb, tbase + TM_SFV + 4 * kb, acc);
-                mma_fp4(tbase + TM_L, pd, make_sdesc(smem_u32(s.ones) + 32 * kb, 512, 16, 4), idesc_fp4(128, 16),
-                        tbase + TM_SFP + 4 * kb, tbase + TM_SF1, acc);
-            }
-            tc_commit(&s.mma_bar);
-        }
-        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
-        mma_phase ^= 1;
-        tc_fence_after();
-        has_f = true;
-    }
-
-    // ---- epilogue: out = (O g_V / 2688 + O_b) / (l / 2688 + l_b)
-    const float lf = has_f ? tmem_ld1_sync(tbase + lane_off + TM_L) * (1.0f / 2688.0f) : 0.0f;
-    const float ltot = lf + (MIXED ? lb : 0.0f);
-    const float sf = has_f ? p.v_g[0] * (1.0f / 2688.0f) / ltot : 0.0f;
-    const float sb = 1.0f / ltot;
-    float* orow = p.out + ((size_t)bh * p.N + row) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; c++) {
-        float o[32], ob[32];
-        if (has_f) {
-            tmem_ld32(tbase + lane_off + TM_O + 32 * c, o);
-            tmem_wait_ld();
-            reg_fence(o);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; i++) o[i] = 0.0f;
-        }
-        if (MIXED && has_b) {
-            tmem_ld32(tbase + lane_off + TM_OB + 32 * c, ob);
-            tmem_wait_ld();
-            reg_fence(ob);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; i++) ob[i] = 0.0f;
-        }
-        if (row < p.N) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(orow + 32 * c + i) =
-                    make_float4(fmaf(o[i], sf, ob[i] * sb), fmaf(o[i + 1], sf, ob[i + 1] * sb),
-                                fmaf(o[i + 2], sf, ob[i + 2] * sb), fmaf(o[i + 3], sf, ob[i + 3] * sb));
-        }
-    }
-    if (p.lse && row < p.N) p.lse[(size_t)bh * p.N + row] = m2 * kLn2 + logf(ltot);
-    return true;
-}
-
-template <int D, bool MIXED>
-__global__ void __launch_bounds__(128, 1) attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                          const __grid_constant__ CUtensorMap tm_k,
-                                                          const __grid_constant__ CUtensorMap tm_v,
-                                                          const __grid_constant__ CUtensorMap tm_qb,
-                                                          const __grid_constant__ CUtensorMap tm_kb,
-                                                          const __grid_constant__ CUtensorMap tm_vb,
-                                                          const AttnParams p)
-{
-    extern __shared__ uint8_t smem_raw[];
-    AttnSmem<D>& s = *reinterpret_cast<AttnSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                     ~(uintptr_t)1023);
-    MixedSmem<D>* mx = MIXED ? reinterpret_cast<MixedSmem<D>*>(reinterpret_cast<uint8_t*>(&s) +
-                                                              ((sizeof(AttnSmem<D>) + 1023) & ~(size_t)1023))
-                             : nullptr;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int t = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // long rows first
-    const int bh = blockIdx.z * p.H + blockIdx.y;
-
-    if (warp == 0) {
-        tmem_alloc(&s.tmem_slot, 512);
-        tmem_relinquish();
-    }
-    if (tid == 0) {
-        mbar_init(&s.tma_bar, 1);
-        mbar_init(&s.mma_bar, 1);
-        fence_mbar_init();
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-    }
-    // constant operand for the row sums: E2M1 1.0 (code 2) with E4M3 scale 1.0
-    for (int i = tid; i < 16 * 64 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.ones)[i] = 0x22222222u;
-    for (int i = tid; i < 512 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(s.onesf)[i] = 0x38383838u;
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tbase = s.tmem_slot;
-
-    if (!attn_body<D, MIXED>(s, mx, &tm_q, &tm_k, &tm_v, &tm_qb, &tm_kb, &tm_vb, p, t, bh, tbase) && tid == 0)
-        sa_raise(SA_ERR_TIMEOUT);
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
 }  // namespace sa

@@ -1,84 +1,135 @@
-// attn_pp.cuh -- NVFP4 attention forward, two query tiles per work item,
-// persistent CTAs.
+// attn_pp.cuh -- NVFP4 attention forward (prefill): persistent CTAs, two
+// query tiles per work item, two softmax threads per query row, optional
+// bf16 blocks inside the same online softmax.
 //
-// Same mathematics and schedule as attn.cuh ("Search Your Block Floating
-// Point Scales!", "ScaleSearchAttention / native NVFP4 execution": Q K^T and
-// P V as block-scaled FP4 tensor-core MMAs with FP32 accumulation; online
-// softmax over key tiles of 128; P requantised per 16 keys with scale 1/2688).
+// "Search Your Block Floating Point Scales!", "ScaleSearchAttention / native
+// NVFP4 execution": Q K^T and P V as block-scaled FP4 tensor-core MMAs with
+// FP32 accumulation; online softmax over key tiles of 128; P requantised per
+// 16 keys with the fixed second-level scale 1/2688.  "ThriftAttention": where
+// the block mask is set, the block's Q K^T and P V run on the raw bf16 inputs
+// (kind::f16 MMAs) inside the same softmax.
 //
 // A work item is (b, h, pair): tile A (query rows 256p..256p+127) and tile B
 // (the next 128).  Each K/V tile is loaded once for both.  The grid holds one
 // CTA per SM; CTA c takes items c, 2G-1-c, 2G+c, ... of the list ordered
-// heaviest causal pair first (a zigzag that evens the per-CTA work).
-//   warp 0        TMA producer: Q tiles (double-buffered across items) and
-//                 a K/V ring whose stages run on across items.
-//   warp 1        MMA issuer (one lane).
-//   warps 4..7    softmax of tile A: one thread per query row (TMEM lane).
-//   warps 8..11   softmax of tile B.
-// The two softmax warpgroups never wait on each other: on each SMSP one warp
-// of A and one of B run independently, so the special-function work of one
-// overlaps the loads, reductions and TMEM traffic of the other.  Across items
-// the next item's loads and first Q K^T proceed while the softmax warps write
-// the previous item's output.
+// heaviest causal pair first.
+//   warp 0        producer (one lane): Q tiles, a ring of NVFP4 K/V stages
+//                 and, with bf16 blocks, the raw K, V and Q tiles they need.
+//   warp 1        Q K^T issuer (one lane).
+//   warp 2        P V issuer (one lane): the two MMA streams wait on different
+//                 events, so a new S is issued the moment its buffer is free
+//                 rather than behind a P V (and each issuer shares its SM
+//                 sub-partition's issue slots with four softmax warps).
+//   warp 3        idle (it keeps five warps on every SM sub-partition, whose
+//                 register files set the launch allocation).
+//   warps 4..11   softmax of tile A, warps 12..19 of tile B: warp w reads the
+//                 TMEM lane quadrant w % 4 (query rows 32(w%4)..+31) and the
+//                 key half h = ((w - 4) / 4) % 2 (columns 64h..64h+63).  The
+//                 two halves of a row meet once per key tile, through shared
+//                 memory and a 64-thread named barrier, to agree on the row
+//                 max; each half then computes its four 16-key block scales
+//                 (one 32-bit scale word of P), its 64 codes and the rescale
+//                 of its half of [O | l].
+// Every SM sub-partition (warps w with equal w % 4) runs two softmax warps of
+// each tile, so the special-function
+// work of one overlaps the TMEM traffic, reductions and waits of the others.
 //
-// TMEM: one S buffer (128 columns) shared by the two tiles and handed back and
-// forth: Q_A K_u^T -> A loads S -> Q_B K_u^T -> B loads S -> Q_A K_{u+1}^T ...
-// plus [O_x | l_x] for each tile and the scale factors (472 of 512 columns).
-// The row sum l accumulates the same dequantised P as O: the V operand of
-// P V carries 16 extra rows of E2M1 1.0 (scale 1.0) after row 127, so column
-// 128 of [O_x | l_x] is l (for D = 64, rows 64..127 of the operand are zero).
-// The softmax warps write P's block scales straight into TMEM.  Every barrier
-// phase is counted over the CTA's whole item sequence.
+// TMEM (512 columns): one S buffer (128) handed between the tiles
+// (Q_A K_u^T -> A reads -> Q_B K_u^T -> B reads -> Q_A K_{u+1}^T ...), the
+// accumulators [O_x | l_x] (144 each; the V operand carries 16 rows of E2M1
+// 1.0 after row 127, so column 128 sums the dequantised P exactly) and the
+// scale factors.  bf16 blocks accumulate into the same O_x: their P, rounded
+// to bf16, is scaled by 2688 / g_V (the ratio between the NVFP4 accumulator's
+// units and raw-V units) and rounded to bf16 again; their row sums stay in
+// registers.
+// Every barrier phase is counted over the CTA's whole item sequence.
 #pragma once
 
 #include "attn.cuh"
 
 namespace sa {
 
-constexpr int kPpStages = 4;
-constexpr int kPpThreads = 384;
+constexpr int kPpThreads = 640;  // 20 warps
+constexpr int kPpStagesF = 4;  // NVFP4 K/V ring of the all-NVFP4 kernel
+constexpr int kPpStagesM = 3;  // ... of the kernel with bf16 blocks
 
-template <int D>
+template <int D, bool MIXED>
 struct PpSmem {
-    alignas(1024) uint8_t q[2][2][128 * D / 2];  // [item % 2][tile]
-    alignas(1024) uint8_t k[kPpStages][128 * D / 2];
-    alignas(1024) uint8_t v[kPpStages][128 * 64 + 16 * 64];  // V^T (D rows), zero rows to 128, 16 rows of 1.0
-    alignas(1024) uint8_t p[2][128 * 64];
-    alignas(16) uint8_t qsf[2][2][D / 64 * 512];
-    uint8_t ksf[kPpStages][D / 64 * 512];
-    uint8_t vsf[kPpStages][2 * 512];
-    float lg2sc[128];  // log2 of each nonzero E4M3 scale value: exponent + log2 of the significand
-    uint64_t q_full[2];   // [item % 2]: Q tiles and scale atoms landed
-    uint64_t q_empty[2];  // [item % 2]: every Q K^T of the item completed
-    uint64_t kv_full[kPpStages];
-    uint64_t kv_empty[kPpStages];
+    static constexpr int S = MIXED ? kPpStagesM : kPpStagesF;
+    static constexpr int QB = MIXED ? 1 : 2;            // Q buffers (items in flight)
+    static constexpr int RB = MIXED ? D / 64 : 1;        // 64-channel regions of a raw bf16 tile
+    static constexpr int RBYTES = MIXED ? 16384 : 1024;  // 128 rows x 128 bytes, 128-byte swizzle
+    alignas(1024) uint8_t q[QB][2][128 * D / 2];
+    alignas(1024) uint8_t k[S][128 * D / 2];
+    alignas(1024) uint8_t v[S][128 * 64 + 16 * 64];  // V^T (D rows), zero rows to 128, 16 rows of 1.0
+    alignas(1024) uint8_t p[2][128 * 64];            // NVFP4 P of each tile; epilogue staging
+    alignas(1024) uint8_t qb[RB][RBYTES];            // raw bf16 Q of one query tile
+    alignas(1024) uint8_t kb[RB][RBYTES];            // raw bf16 K tile (K-major)
+    alignas(1024) uint8_t vb[RB][RBYTES];            // raw bf16 V tile (rows = keys, MN-major operand)
+    alignas(1024) uint8_t pb[2][RBYTES];             // bf16 P of one query tile: 2 x 64 keys
+    alignas(16) uint8_t qsf[QB][2][D / 64 * 512];
+    uint8_t ksf[S][D / 64 * 512];
+    uint8_t vsf[S][2 * 512];
+    float lg2sc[128];         // log2 of each nonzero E4M3 scale value
+    float xch[2][2][2][128];  // half-row exchange: [use parity][tile][half][row]
+    uint64_t q_full[QB];      // Q tiles and scale atoms landed
+    uint64_t q_empty[QB];     // every Q K^T of the item completed
+    uint64_t kv_full[S];
+    uint64_t kv_empty[S];
     uint64_t s_full[2];  // [tile]: S holds this tile's scores
-    uint64_t s_free[2];  // [tile]: this tile's warps have read S
-    uint64_t p_full[2];
-    uint64_t o_done[2];
+    uint64_t s_free[2];  // [tile]: this tile's 8 warps have read S
+    uint64_t p_full[2];  // [tile]: this tile's 8 warps wrote P and rescaled O
+    uint64_t o_done[2];  // [tile]: the tile's P V completed
+    uint64_t xbar[2][4]; // [tile][quadrant]: both halves of the rows posted their value
+    uint64_t drain;      // both issuers' tensor-core work has completed (kernel exit)
+    // bf16 blocks: raw K / V tiles (one per key tile that has a bf16 block),
+    // raw Q tiles (reloaded when the next bf16 block is another query tile's:
+    // qb_empty completes once per reload) and the bf16 P buffer, shared by the
+    // two tiles one block at a time (pb_grant[x] completes once per bf16 block
+    // of tile x, when the block before it has finished its P V).  Each phase
+    // of every barrier is awaited in order by its waiters, as parity waits need.
+    uint64_t kb_full, kb_empty, vb_full, vb_empty, qb_full, qb_empty, pb_grant[2];
     uint32_t tmem_slot;
     int abort;
 };
 
-// TMEM columns
 // TMEM columns: [O_x | l_x] is PP_OW wide at PP_O + PP_OW x (l in column 128);
-// SFV: 64-key block kb at + 8 kb (V rows in + 0..3, the 1.0 rows' scale at + 4);
-// SFP: tile x at + 8 x, block kb at + 4 kb.
+// SFQ: tile x at + 8 x; SFV: 64-key block kb at + 8 kb (V rows in + 0..3, the
+// 1.0 rows' scale at + 4); SFP: tile x at + 8 x, block kb at + 4 kb.
+constexpr int PP_REG_CTL = 64, PP_REG_SM = 104;  // 128 x 64 + 512 x 104 = 640 x 96
+static_assert(128 * PP_REG_CTL + 512 * PP_REG_SM <= kPpThreads * 96, "register split exceeds the launch allocation");
 constexpr uint32_t PP_S = 0, PP_O = 128, PP_OW = 144, PP_SFQ = 416, PP_SFK = 432, PP_SFV = 440, PP_SFP = 456;
 
-SA_DEV bool pp_wait(uint64_t* bar, uint32_t parity, volatile int* abort)
+// Bounded wait for the phase of `bar` with the given parity.  Gives up (false)
+// when another role has aborted, or after `lim` cycles, when it records
+// SA_ERR_TIMEOUT and raises the CTA's abort flag so every role unwinds.
+SA_DEV bool pp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long lim)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
+    const uint32_t hint = (uint32_t)min(max(lim / 4, 32LL), 1000000LL);  // ns, below the limit in cycles
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_hint(bar, parity, hint)) {
         if (*abort) return false;
-        if (clock64() - t0 > SA_WAIT_CYCLES) {
+        if (clock64() - t0 > lim) {
             *abort = 1;
             sa_raise(SA_ERR_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+// Wait (bounded by the library default) for a phase the caller knows will
+// complete: the copies and tensor-core work a role issued, drained before the
+// CTA releases its shared memory and tensor memory.
+SA_DEV void pp_drain(uint64_t* bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > SA_WAIT_CYCLES) {
+            sa_raise(SA_ERR_TIMEOUT);
+            return;
+        }
 }
 
 SA_DEV float pp_max3(float a, float b, float c)
@@ -107,12 +158,13 @@ SA_DEV void pp_setmaxnreg_dec()
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Work item of the zigzag schedule: round j of this CTA, or -1 past the end.
+// Work item of the zigzag schedule.
 struct PpItem {
     int bh, pair, nuA, nuB, nu;
     bool hasB;
 };
 
+// Item index of round j of this CTA, or -1 past the end.
 SA_DEV int pp_item_index(int j, int nitems)
 {
     const int G = gridDim.x;
@@ -137,22 +189,187 @@ SA_DEV PpItem pp_item(const AttnParams& p, int i)
     return it;
 }
 
-template <int D>
+// Is the block (query tile x of the item, key tile u) a bf16 block?
+template <bool MIXED>
+SA_DEV bool pp_bf16(const AttnParams& p, const PpItem& I, int x, int u)
+{
+    if (!MIXED) return false;
+    if (u >= (x ? I.nuB : I.nuA)) return false;
+    return __ldg(p.mask + ((size_t)I.bh * p.T + 2 * I.pair + x) * p.T + u) != 0;
+}
+
+// bf16 flags of key tiles [base, base + 32) of an item's two query tiles, read
+// from the mask once per 32 tiles instead of per tile.
+struct PpFlags {
+    int base;
+    uint32_t a, b;
+};
+
+// 16 mask bytes -> 16 bits (bit i set when byte i is nonzero).
+SA_DEV uint32_t pp_bytes_to_bits(uint4 w)
+{
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+    uint32_t bits = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t nz = __vcmpne4(v[i], 0u) & 0x01010101u;  // one bit per nonzero byte, at bit 8j
+        bits |= ((nz * 0x01020408u) >> 24) << (4 * i);         // gather bits 0, 8, 16, 24 to 0..3
+    }
+    return bits;
+}
+
+template <bool MIXED>
+SA_DEV void pp_flags_fill(PpFlags& f, const AttnParams& p, const PpItem& I, int base)
+{
+    f.base = base;
+    f.a = f.b = 0;
+    if (!MIXED) return;
+    const uint8_t* ra = p.mask + ((size_t)I.bh * p.T + 2 * I.pair) * p.T + base;
+    const uint8_t* rb = ra + p.T;
+    if ((p.T & 15) == 0 && base + 32 <= p.T) {
+        f.a = pp_bytes_to_bits(__ldg(reinterpret_cast<const uint4*>(ra))) |
+              (pp_bytes_to_bits(__ldg(reinterpret_cast<const uint4*>(ra + 16))) << 16);
+        if (I.hasB)
+            f.b = pp_bytes_to_bits(__ldg(reinterpret_cast<const uint4*>(rb))) |
+                  (pp_bytes_to_bits(__ldg(reinterpret_cast<const uint4*>(rb + 16))) << 16);
+    } else {
+        for (int i = 0; i < 32 && base + i < p.T; i++) {
+            f.a |= (uint32_t)(__ldg(ra + i) != 0) << i;
+            if (I.hasB) f.b |= (uint32_t)(__ldg(rb + i) != 0) << i;
+        }
+    }
+    // only key tiles the query tile visits count
+    const int na = I.nuA - base, nb = I.nuB - base;
+    f.a &= na >= 32 ? ~0u : (na <= 0 ? 0u : (1u << na) - 1u);
+    f.b &= nb >= 32 ? ~0u : (nb <= 0 ? 0u : (1u << nb) - 1u);
+}
+
+// bf16 flags of key tile u for query tiles A (bit 0) and B (bit 1).
+template <bool MIXED>
+SA_DEV uint32_t pp_flags(PpFlags& f, const AttnParams& p, const PpItem& I, int u)
+{
+    if (!MIXED) return 0;
+    if (u < f.base || u >= f.base + 32) pp_flags_fill<MIXED>(f, p, I, u & ~31);
+    const int i = u - f.base;
+    return ((f.a >> i) & 1u) | (((f.b >> i) & 1u) << 1);
+}
+
+// Position of the producer's walk over this CTA's items and their key tiles.
+struct PpCursor {
+    int j;   // round
+    int it;  // items passed
+    int i;   // item index, -1 past the end
+    int u;   // key tile
+    int x;   // query tile (event walks)
+    PpItem I;
+};
+
+SA_DEV void pp_cursor_seek_item(PpCursor& c, const AttnParams& p, int nitems, int nrounds)
+{
+    c.i = -1;
+    for (; c.j < nrounds; c.j++) {
+        c.i = pp_item_index(c.j, nitems);
+        if (c.i >= 0) {
+            c.I = pp_item(p, c.i);
+            return;
+        }
+    }
+    c.i = -1;
+}
+
+SA_DEV void pp_cursor_next_item(PpCursor& c, const AttnParams& p, int nitems, int nrounds)
+{
+    c.j++;
+    c.it++;
+    c.u = 0;
+    c.x = 0;
+    pp_cursor_seek_item(c, p, nitems, nrounds);
+}
+
+// Could any of the 16 key tiles u0..u0+15 of the item hold a bf16 block?  (A
+// cheap skip for the long runs of NVFP4 tiles: one 16-byte load per mask row
+// when the rows are 16-byte aligned; false means certainly not.)
+template <bool MIXED>
+SA_DEV bool pp_maybe_bf16_x16(const AttnParams& p, const PpItem& I, int u0)
+{
+    if (!MIXED) return false;
+    if ((p.T & 15) || u0 + 16 > p.T) return true;
+    const uint8_t* row = p.mask + ((size_t)I.bh * p.T + 2 * I.pair) * p.T + u0;
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(row));
+    uint32_t any = a.x | a.y | a.z | a.w;
+    if (I.hasB) {
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(row + p.T));
+        any |= b.x | b.y | b.z | b.w;
+    }
+    return any != 0;
+}
+
+// Advance to the first key tile at or after c.u (crossing items) that holds a
+// bf16 block of either query tile.  At most `budget` probes per call: returns
+// 1 (found), 0 (not yet: call again) or -1 (past the end).
+template <bool MIXED>
+SA_DEV int pp_next_bf16_tile(PpCursor& c, const AttnParams& p, int nitems, int nrounds, int budget)
+{
+    while (c.i >= 0) {
+        while (c.u < c.I.nu) {
+            if (budget-- <= 0) return 0;
+            if ((c.u & 15) == 0 && !pp_maybe_bf16_x16<MIXED>(p, c.I, c.u)) {
+                c.u += 16;
+                continue;
+            }
+            if (pp_bf16<MIXED>(p, c.I, 0, c.u) || pp_bf16<MIXED>(p, c.I, 1, c.u)) return 1;
+            c.u++;
+        }
+        pp_cursor_next_item(c, p, nitems, nrounds);
+    }
+    return -1;
+}
+
+// Advance to the first bf16 block (x, u) at or after (c.u, c.x) in the order
+// u ascending, then x (the issue order of Q K^T and of P V); budget and
+// return value as pp_next_bf16_tile.
+template <bool MIXED>
+SA_DEV int pp_next_bf16_block(PpCursor& c, const AttnParams& p, int nitems, int nrounds, int budget)
+{
+    while (c.i >= 0) {
+        while (c.u < c.I.nu) {
+            if (budget-- <= 0) return 0;
+            if (c.x == 0 && (c.u & 15) == 0 && !pp_maybe_bf16_x16<MIXED>(p, c.I, c.u)) {
+                c.u += 16;
+                continue;
+            }
+            for (; c.x < 2; c.x++)
+                if (pp_bf16<MIXED>(p, c.I, c.x, c.u)) return 1;
+            c.x = 0;
+            c.u++;
+        }
+        pp_cursor_next_item(c, p, nitems, nrounds);
+    }
+    return -1;
+}
+
+template <int D, bool MIXED>
 __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                     const __grid_constant__ CUtensorMap tm_k,
                                                                     const __grid_constant__ CUtensorMap tm_v,
+                                                                    const __grid_constant__ CUtensorMap tm_qb,
+                                                                    const __grid_constant__ CUtensorMap tm_kb,
+                                                                    const __grid_constant__ CUtensorMap tm_vb,
                                                                     const AttnParams p)
 {
+    using Sm = PpSmem<D, MIXED>;
+    constexpr int S = Sm::S, QB = Sm::QB;
     constexpr int KB = D / 64;
+    constexpr int HD = D / 2;  // O columns of one softmax half
     constexpr uint32_t QSW = D == 128 ? 4u : 6u;
     constexpr uint32_t QSBO = 8 * D / 2;
     extern __shared__ uint8_t smem_raw[];
-    PpSmem<D>& s = *reinterpret_cast<PpSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                 ~(uintptr_t)1023);
+    Sm& s = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nitems = p.B * p.H * ((p.T + 1) / 2);
     const int nrounds = (nitems + (int)gridDim.x - 1) / (int)gridDim.x;
     volatile int* abort = &s.abort;
+    const long long lim = p.wait_cycles;
 
     if (warp == 0) {
         tmem_alloc(&s.tmem_slot, 512);
@@ -160,24 +377,41 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
     }
     if (tid == 0) {
         s.abort = 0;
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < QB; i++) {
             mbar_init(&s.q_full[i], 1);
             mbar_init(&s.q_empty[i], 1);
         }
-        for (int i = 0; i < kPpStages; i++) {
+        for (int i = 0; i < S; i++) {
             mbar_init(&s.kv_full[i], 1);
-            mbar_init(&s.kv_empty[i], 1);
+            mbar_init(&s.kv_empty[i], 2);  // released by both issuers
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(&s.s_full[i], 1);
-            mbar_init(&s.s_free[i], 4);
-            mbar_init(&s.p_full[i], 4);
+            mbar_init(&s.s_free[i], 8);
+            mbar_init(&s.p_full[i], 8);
             mbar_init(&s.o_done[i], 1);
+            for (int q = 0; q < 4; q++) mbar_init(&s.xbar[i][q], 2);
         }
+        if (MIXED) {
+            mbar_init(&s.kb_full, 1);
+            mbar_init(&s.kb_empty, 1);
+            mbar_init(&s.vb_full, 1);
+            mbar_init(&s.vb_empty, 1);
+            mbar_init(&s.qb_full, 1);
+            mbar_init(&s.qb_empty, 1);
+            mbar_init(&s.pb_grant[0], 1);
+            mbar_init(&s.pb_grant[1], 1);
+        }
+        mbar_init(&s.drain, 2);  // both issuers
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        if (MIXED) {
+            tma_prefetch_desc(&tm_qb);
+            tma_prefetch_desc(&tm_kb);
+            tma_prefetch_desc(&tm_vb);
+        }
     }
     if (tid < 128) {
         // (e - 7) + log2(1 + m/8) for normal bytes, -7 + log2(m/4) for subnormal ones
@@ -186,7 +420,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
         s.lg2sc[tid] = (e ? (float)((int)e - 7) : -7.0f) + sig;
     }
     // rows D..127 of every V stage are zero, rows 128..143 are E2M1 1.0
-    for (int i = tid; i < kPpStages * (144 - D) * 16; i += blockDim.x) {
+    for (int i = tid; i < S * (144 - D) * 16; i += blockDim.x) {
         const int st = i / ((144 - D) * 16), w = i % ((144 - D) * 16);
         reinterpret_cast<uint32_t*>(s.v[st] + D * 64)[w] = w >= (128 - D) * 16 ? 0x22222222u : 0u;
     }
@@ -208,249 +442,509 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
     __syncthreads();
     tc_fence_after();
 
-    if (warp < 4) pp_setmaxnreg_dec<40>();
+    // register split: 128 x PP_REG_CTL + 512 x PP_REG_SM <= 640 x 96, the launch
+    // allocation (five warps per SM sub-partition cap it at 96 per thread)
+    if (warp < 4) pp_setmaxnreg_dec<PP_REG_CTL>();
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ producer
+        // Independent streams, each in its own order, polled in turn so that
+        // none blocks another: (Q) NVFP4 Q tiles of each item, (R) the NVFP4
+        // K/V ring; with bf16 blocks (K) raw K tiles, (V) raw V tiles and
+        // (B) raw Q tiles.
         if (lane == 0) {
-            bool ok = true;
-            int g = 0;   // K/V tiles loaded so far (ring position)
-            int it = 0;  // items of this CTA so far
-            for (int j = 0; ok && j < nrounds; j++) {
-                const int i = pp_item_index(j, nitems);
-                if (i < 0) continue;
-                const PpItem I = pp_item(p, i);
-                const int qs = it & 1;
-                // Q buffers of this parity are free once the item two back issued its last Q K^T
-                if (it >= 2 && !pp_wait(&s.q_empty[qs], ((it >> 1) - 1) & 1, abort)) break;
-                const int nq = I.hasB ? 2 : 1;
-                mbar_expect_tx(&s.q_full[qs], nq * (128 * D / 2 + KB * 512));
-                for (int x = 0; x < nq; x++) {
-                    const int tt = 2 * I.pair + x;
-                    tma_load_3d(s.q[qs][x], &tm_q, &s.q_full[qs], 0, tt * 128, I.bh);
-                    bulk_load(s.qsf[qs][x], p.q_sf + ((size_t)I.bh * p.T + tt) * KB * 512, KB * 512, &s.q_full[qs]);
+            PpCursor cf{}, cr{};  // streams Q and R
+            pp_cursor_seek_item(cf, p, nitems, nrounds);
+            cr = cf;
+            int rg = 0;  // K/V tiles loaded so far (ring position)
+            int nqf[QB] = {};  // Q loads per Q buffer
+            // bf16 streams: state 1 = at the next bf16 tile (block), 0 = still
+            // scanning the mask (a few probes per poll), -1 = past the end
+            PpCursor ck{}, cv{}, cq{};
+            int kst = -1, vst = -1, qst = -1;
+            int nk = 0, nv = 0, nrl = 0, qhold = -1;  // raw K, V tiles and raw Q reloads issued
+            if (MIXED) {
+                ck = cf;
+                cv = cf;
+                cq = cf;
+                kst = vst = qst = 0;
+            }
+            long long t_last = clock64();
+            while (cf.i >= 0 || cr.i >= 0 || kst >= 0 || vst >= 0 || qst >= 0) {
+                bool prog = false;
+                if (cf.i >= 0) {
+                    const PpItem& I = cf.I;
+                    const int qs = cf.it % QB;
+                    // Q buffers are free once the item QB back issued its last Q K^T
+                    if (cf.it < QB || mbar_test(&s.q_empty[qs], ((cf.it / QB) - 1) & 1)) {
+                        const int nq = I.hasB ? 2 : 1;
+                        mbar_expect_tx(&s.q_full[qs], nq * (128 * D / 2 + KB * 512));
+                        for (int x = 0; x < nq; x++) {
+                            const int tt = 2 * I.pair + x;
+                            tma_load_3d(s.q[qs][x], &tm_q, &s.q_full[qs], 0, tt * 128, I.bh);
+                            bulk_load(s.qsf[qs][x], p.q_sf + ((size_t)I.bh * p.T + tt) * KB * 512, KB * 512,
+                                      &s.q_full[qs]);
+                        }
+                        nqf[qs]++;
+                        pp_cursor_next_item(cf, p, nitems, nrounds);
+                        prog = true;
+                    }
                 }
-                for (int u = 0; u < I.nu; u++, g++) {
-                    const int st = g % kPpStages;
-                    if (g >= kPpStages && !pp_wait(&s.kv_empty[st], ((g / kPpStages) & 1) ^ 1, abort)) {
-                        ok = false;
+                if (cr.i >= 0) {
+                    const PpItem& I = cr.I;
+                    const int st = rg % S, u = cr.u;
+                    if (rg < S || mbar_test(&s.kv_empty[st], ((rg / S) & 1) ^ 1)) {
+                        const int nk2 = min(128, p.N - u * 128);
+                        const int kblocks = nk2 > 64 ? 2 : 1;
+                        mbar_expect_tx(&s.kv_full[st], 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
+                        tma_load_3d(s.k[st], &tm_k, &s.kv_full[st], 0, u * 128, I.bh);
+                        bulk_load(s.ksf[st], p.k_sf + ((size_t)I.bh * p.T + u) * KB * 512, KB * 512,
+                                  &s.kv_full[st]);
+                        tma_load_3d(s.v[st], &tm_v, &s.kv_full[st], 0, u * D, I.bh);
+                        bulk_load(s.vsf[st], p.v_sf + ((size_t)I.bh * p.CKv + 2 * u) * 512, kblocks * 512,
+                                  &s.kv_full[st]);
+                        rg++;
+                        prog = true;
+                        if (++cr.u == I.nu) pp_cursor_next_item(cr, p, nitems, nrounds);
+                    }
+                }
+                if (MIXED) {
+                    constexpr int kProbe = 8;  // mask probes per stream and poll
+                    if (kst == 0 && (kst = pp_next_bf16_tile<MIXED>(ck, p, nitems, nrounds, kProbe)) >= 0) prog = true;
+                    if (vst == 0 && (vst = pp_next_bf16_tile<MIXED>(cv, p, nitems, nrounds, kProbe)) >= 0) prog = true;
+                    if (qst == 0 && (qst = pp_next_bf16_block<MIXED>(cq, p, nitems, nrounds, kProbe)) >= 0) prog = true;
+                    // raw K of bf16 key tile nk: the previous one's Q K^T have completed
+                    if (kst == 1 && (nk == 0 || mbar_test(&s.kb_empty, (nk - 1) & 1))) {
+                        mbar_expect_tx(&s.kb_full, 128 * D * 2);
+                        for (int r = 0; r < D / 64; r++)
+                            tma_load_3d(s.kb[r], &tm_kb, &s.kb_full, 64 * r, ck.u * 128, ck.I.bh);
+                        nk++;
+                        ck.u++;
+                        kst = 0;
+                        prog = true;
+                    }
+                    // raw V of bf16 key tile nv: the previous one's P V have completed
+                    if (vst == 1 && (nv == 0 || mbar_test(&s.vb_empty, (nv - 1) & 1))) {
+                        mbar_expect_tx(&s.vb_full, 128 * D * 2);
+                        for (int r = 0; r < D / 64; r++)
+                            tma_load_3d(s.vb[r], &tm_vb, &s.vb_full, 64 * r, cv.u * 128, cv.I.bh);
+                        nv++;
+                        cv.u++;
+                        vst = 0;
+                        prog = true;
+                    }
+                    // raw Q for the next bf16 block: reload when it is another query
+                    // tile's, once the issuer has released the buffer (one qb_empty
+                    // phase per reload)
+                    if (qst == 1) {
+                        const int want = cq.it * 2 + cq.x;
+                        bool go = want == qhold;
+                        if (!go && (nrl == 0 || mbar_test(&s.qb_empty, (nrl - 1) & 1))) {
+                            mbar_expect_tx(&s.qb_full, 128 * D * 2);
+                            for (int r = 0; r < D / 64; r++)
+                                tma_load_3d(s.qb[r], &tm_qb, &s.qb_full, 64 * r, (2 * cq.I.pair + cq.x) * 128,
+                                            cq.I.bh);
+                            qhold = want;
+                            nrl++;
+                            go = true;
+                        }
+                        if (go) {
+                            if (++cq.x == 2) {
+                                cq.x = 0;
+                                cq.u++;
+                            }
+                            qst = 0;
+                            prog = true;
+                        }
+                    }
+                }
+                if (prog) {
+                    t_last = clock64();
+                } else {
+                    if (*abort) break;
+                    if (clock64() - t_last > lim) {
+                        *abort = 1;
+                        sa_raise(SA_ERR_TIMEOUT);
                         break;
                     }
-                    const int nk = min(128, p.N - u * 128);
-                    const int kblocks = nk > 64 ? 2 : 1;
-                    mbar_expect_tx(&s.kv_full[st], 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
-                    tma_load_3d(s.k[st], &tm_k, &s.kv_full[st], 0, u * 128, I.bh);
-                    bulk_load(s.ksf[st], p.k_sf + ((size_t)I.bh * p.T + u) * KB * 512, KB * 512, &s.kv_full[st]);
-                    tma_load_3d(s.v[st], &tm_v, &s.kv_full[st], 0, u * D, I.bh);
-                    bulk_load(s.vsf[st], p.v_sf + ((size_t)I.bh * p.CKv + 2 * u) * 512, kblocks * 512,
-                              &s.kv_full[st]);
                 }
-                it++;
+            }
+            // every copy issued has landed before the CTA releases its shared memory
+            // (after an abort too): wait for each barrier's last issued phase
+            for (int b = 0; b < QB; b++)
+                if (nqf[b] > 0) pp_drain(&s.q_full[b], (nqf[b] - 1) & 1);
+            for (int st = 0; st < S; st++) {
+                const int c = (rg - st + S - 1) / S;  // loads into stage st
+                if (c > 0) pp_drain(&s.kv_full[st], (c - 1) & 1);
+            }
+            if (MIXED) {
+                if (nk > 0) pp_drain(&s.kb_full, (nk - 1) & 1);
+                if (nv > 0) pp_drain(&s.vb_full, (nv - 1) & 1);
+                if (nrl > 0) pp_drain(&s.qb_full, (nrl - 1) & 1);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+        // ------------------------------------------------ Q K^T issuer (one lane)
+        // Key tiles in order; per tile Q_A K_u^T then Q_B K_u^T into the shared S
+        // buffer, each once the previous S has been read.  Descriptors are bases
+        // plus byte offsets / 16 (the address field of a shared-memory descriptor).
         if (lane == 0) {
+            const uint64_t dq0 = make_sdesc(smem_u32(&s.q[0][0][0]), QSBO, 16, QSW);
+            const uint64_t dk0 = make_sdesc(smem_u32(&s.k[0][0]), QSBO, 16, QSW);
+            const uint32_t idq = idesc_fp4(128, 128);
             bool ok = true;
             int g0 = 0;  // ring position of the current item's key tile 0
-            int kv_waited = -1, sfk_tile = -1, last_x = -1, last_idx = -1;
-            int nS[2] = {0, 0}, nP[2] = {0, 0};  // Q_x K^T and P_x V issued so far
+            int last_x = -1, last_idx = -1;
+            int nS[2] = {0, 0};
             int it = 0;
+            int bk = 0, bq = 0, qhold = -1;  // bf16: raw K tiles and raw Q loads used so far
             for (int j = 0; ok && j < nrounds; j++) {
                 const int i = pp_item_index(j, nitems);
                 if (i < 0) continue;
                 const PpItem I = pp_item(p, i);
-                const int qs = it & 1;
-                if (!pp_wait(&s.q_full[qs], (it >> 1) & 1, abort)) break;
+                const int qs = it % QB;
+                if (!pp_wait(&s.q_full[qs], (it / QB) & 1, abort, lim)) break;
                 tc_fence_after();
                 for (int x = 0; x < (I.hasB ? 2 : 1); x++)
                     for (int kb = 0; kb < KB; kb++)
                         tc_cp_sf(tbase + PP_SFQ + 8 * x + 4 * kb, smem_u32(s.qsf[qs][x] + 512 * kb));
-                // Q_x K_u^T into the shared S buffer once its previous reader is done
-                auto qk = [&](int x, int u) -> bool {
-                    const int gt = g0 + u, st = gt % kPpStages;
-                    if (gt > kv_waited) {
-                        if (!pp_wait(&s.kv_full[st], (gt / kPpStages) & 1, abort)) return false;
-                        kv_waited = gt;
-                    }
-                    if (last_x >= 0 && !pp_wait(&s.s_free[last_x], last_idx & 1, abort)) return false;
-                    tc_fence_after();
-                    if (sfk_tile != gt) {
-                        for (int kb = 0; kb < KB; kb++)
-                            tc_cp_sf(tbase + PP_SFK + 4 * kb, smem_u32(s.ksf[st] + 512 * kb));
-                        sfk_tile = gt;
-                    }
-                    for (int kb = 0; kb < KB; kb++)
-                        mma_fp4(tbase + PP_S, make_sdesc(smem_u32(s.q[qs][x]) + 32 * kb, QSBO, 16, QSW),
-                                make_sdesc(smem_u32(s.k[st]) + 32 * kb, QSBO, 16, QSW), idesc_fp4(128, 128),
-                                tbase + PP_SFQ + 8 * x + 4 * kb, tbase + PP_SFK + 4 * kb, kb > 0);
-                    tc_commit(&s.s_full[x]);
-                    last_x = x;
-                    last_idx = nS[x]++;
-                    return true;
-                };
-                // [O_x | l_x] (+)= P_x [V_u | 0 | 1]
-                auto pv = [&](int x, int u) -> bool {
-                    if (!pp_wait(&s.p_full[x], nP[x] & 1, abort)) return false;
-                    tc_fence_after();
-                    const int nk = min(128, p.N - u * 128);
-                    const int kblocks = nk > 64 ? 2 : 1;
-                    const int st = (g0 + u) % kPpStages;
-                    for (int kb = 0; kb < kblocks; kb++) {
-                        const uint64_t pd = make_sdesc(smem_u32(s.p[x]) + 32 * kb, 512, 16, 4);
-                        const uint32_t acc = (u > 0 || kb > 0) ? 1u : 0u;
-                        mma_fp4(tbase + PP_O + PP_OW * x, pd, make_sdesc(smem_u32(s.v[st]) + 32 * kb, 512, 16, 4),
-                                idesc_fp4(128, PP_OW), tbase + PP_SFP + 8 * x + 4 * kb, tbase + PP_SFV + 8 * kb,
-                                acc);
-                    }
-                    tc_commit(&s.o_done[x]);
-                    nP[x]++;
-                    return true;
-                };
-                // Issue order, steady state: P_A V_u, Q_B K_{u+1}^T, P_B V_u, Q_A K_{u+2}^T.
-                // Scores are consumed in the order A0 B0 A1 B1 ...
-                ok = qk(0, 0);
-                if (ok && I.hasB) ok = qk(1, 0);
-                if (ok && I.nuA > 1) ok = qk(0, 1);
+                PpFlags fl{-64, 0, 0};
                 for (int u = 0; ok && u < I.nu; u++) {
-                    const int st = (g0 + u) % kPpStages;
-                    // V scale atoms of key tile u (P V of the tile before was issued earlier)
-                    const int nk = min(128, p.N - u * 128);
-                    const int kblocks = nk > 64 ? 2 : 1;
-                    for (int kb = 0; kb < kblocks; kb++)
-                        tc_cp_sf(tbase + PP_SFV + 8 * kb, smem_u32(s.vsf[st] + 512 * kb));
-                    if (u < I.nuA && !(ok = pv(0, u))) break;
-                    if (u + 1 < I.nuB && !(ok = qk(1, u + 1))) break;
-                    if (u < I.nuB && !(ok = pv(1, u))) break;
-                    tc_commit(&s.kv_empty[st]);
-                    if (u + 2 < I.nuA && !(ok = qk(0, u + 2))) break;
+                    const int gt = g0 + u, st = gt % S;
+                    const uint32_t f = pp_flags<MIXED>(fl, p, I, u);
+                    if (!(ok = pp_wait(&s.kv_full[st], (gt / S) & 1, abort, lim))) break;
+                    bool sfk = false;
+                    for (int x = 0; x < 2; x++) {
+                        if (u >= (x ? I.nuB : I.nuA)) continue;
+                        if (last_x >= 0 && !(ok = pp_wait(&s.s_free[last_x], last_idx & 1, abort, lim))) break;
+                        tc_fence_after();
+                        if (MIXED && ((f >> x) & 1)) {
+                            // bf16 block: S = q.k on the raw tiles (K = 16 per MMA)
+                            if ((x == 0 || !(f & 1)) && !(ok = pp_wait(&s.kb_full, bk & 1, abort, lim))) break;
+                            const int want = it * 2 + x;
+                            if (want != qhold) {
+                                // hand the raw Q buffer back (once the Q K^T issued so far
+                                // complete) and wait for this query tile's
+                                if (qhold >= 0) tc_commit(&s.qb_empty);
+                                if (!(ok = pp_wait(&s.qb_full, bq & 1, abort, lim))) break;
+                                bq++;
+                                qhold = want;
+                            }
+                            tc_fence_after();
+                            for (int ks = 0; ks < D / 16; ks++)
+                                mma_bf16(tbase + PP_S, make_sdesc(smem_u32(s.qb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
+                                         make_sdesc(smem_u32(s.kb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
+                                         idesc_bf16(128, 128, 0), ks > 0);
+                            if (x == 1 || !(f & 2)) {  // last bf16 Q K^T of this key tile
+                                tc_commit(&s.kb_empty);
+                                bk++;
+                            }
+                        } else {
+                            if (!sfk) {
+                                for (int kb = 0; kb < KB; kb++)
+                                    tc_cp_sf(tbase + PP_SFK + 4 * kb, smem_u32(s.ksf[st] + 512 * kb));
+                                sfk = true;
+                            }
+                            const uint64_t dq = dq0 + (uint64_t)(((qs * 2 + x) * (128 * D / 2)) >> 4);
+                            const uint64_t dk = dk0 + (uint64_t)((st * (128 * D / 2)) >> 4);
+#pragma unroll
+                            for (int kb = 0; kb < KB; kb++)
+                                mma_fp4(tbase + PP_S, dq + 2 * kb, dk + 2 * kb, idq, tbase + PP_SFQ + 8 * x + 4 * kb,
+                                        tbase + PP_SFK + 4 * kb, kb > 0);
+                        }
+                        tc_commit(&s.s_full[x]);
+                        last_x = x;
+                        last_idx = nS[x]++;
+                    }
+                    if (!ok) break;
+                    tc_commit(&s.kv_empty[st]);  // this tile's Q K^T are issued (one of two releases)
                 }
                 // every Q K^T of this item has been issued: release its Q buffers
                 if (ok) tc_commit(&s.q_empty[qs]);
                 g0 += I.nu;
                 it++;
             }
+            // every MMA and scale copy issued has completed before TMEM is released
+            tc_commit(&s.drain);
+            pp_drain(&s.drain, 0);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------ P V issuer (one lane)
+        // Key tiles in order; per tile [O_A | l_A] (+)= P_A [V_u | 0 | 1] then the
+        // same for B (or O_x += P_x V_u for a bf16 block), each once its P is in.
+        if (lane == 0) {
+            const uint64_t dp0 = make_sdesc(smem_u32(&s.p[0][0]), 512, 16, 4);
+            const uint64_t dv0 = make_sdesc(smem_u32(&s.v[0][0]), 512, 16, 4);
+            const uint32_t idv = idesc_fp4(128, PP_OW);
+            bool ok = true;
+            int g0 = 0;
+            int nP[2] = {0, 0};
+            int bv = 0;  // bf16: raw V tiles used so far
+            // the next bf16 block after the one being issued (hands the bf16 P buffer on)
+            PpCursor nx{};
+            int nx_st = -1;
+            if (MIXED) {
+                pp_cursor_seek_item(nx, p, nitems, nrounds);
+                nx_st = pp_next_bf16_block<MIXED>(nx, p, nitems, nrounds, 1 << 30);
+                if (nx_st == 1) mbar_arrive(&s.pb_grant[nx.x]);  // the first bf16 block may write P at once
+            }
+            for (int j = 0; ok && j < nrounds; j++) {
+                const int i = pp_item_index(j, nitems);
+                if (i < 0) continue;
+                const PpItem I = pp_item(p, i);
+                PpFlags fl{-64, 0, 0};
+                for (int u = 0; ok && u < I.nu; u++) {
+                    const int gt = g0 + u, st = gt % S;
+                    const uint32_t f = pp_flags<MIXED>(fl, p, I, u);
+                    if (!(ok = pp_wait(&s.kv_full[st], (gt / S) & 1, abort, lim))) break;
+                    tc_fence_after();
+                    // V scale atoms of key tile u (the P V of the tile before was issued earlier)
+                    const int nk = min(128, p.N - u * 128);
+                    const int kblocks = nk > 64 ? 2 : 1;
+                    for (int kb = 0; kb < kblocks; kb++)
+                        tc_cp_sf(tbase + PP_SFV + 8 * kb, smem_u32(s.vsf[st] + 512 * kb));
+                    for (int x = 0; x < 2; x++) {
+                        if (u >= (x ? I.nuB : I.nuA)) continue;
+                        if (!(ok = pp_wait(&s.p_full[x], nP[x] & 1, abort, lim))) break;
+                        tc_fence_after();
+                        if (MIXED && ((f >> x) & 1)) {
+                            if ((x == 0 || !(f & 1)) && !(ok = pp_wait(&s.vb_full, bv & 1, abort, lim))) break;
+                            tc_fence_after();
+                            for (int ks = 0; ks < 8; ks++)
+                                mma_bf16(tbase + PP_O + PP_OW * x,
+                                         make_sdesc(smem_u32(s.pb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
+                                         make_sdesc(smem_u32(s.vb[0]) + 2048 * ks, 1024, 16384, 2),
+                                         idesc_bf16(128, D, 1), (u > 0 || ks > 0) ? 1u : 0u);
+                            // hand the bf16 P buffer to the next bf16 block once this P V completes
+                            if (++nx.x == 2) {
+                                nx.x = 0;
+                                nx.u++;
+                            }
+                            nx_st = pp_next_bf16_block<MIXED>(nx, p, nitems, nrounds, 1 << 30);
+                            if (nx_st == 1) tc_commit(&s.pb_grant[nx.x]);
+                            if (x == 1 || !(f & 2)) {  // last bf16 P V of this key tile
+                                tc_commit(&s.vb_empty);
+                                bv++;
+                            }
+                        } else {
+                            const uint64_t dp = dp0 + (uint64_t)((x * (128 * 64)) >> 4);
+                            const uint64_t dv = dv0 + (uint64_t)((st * (128 * 64 + 16 * 64)) >> 4);
+                            for (int kb = 0; kb < kblocks; kb++)
+                                mma_fp4(tbase + PP_O + PP_OW * x, dp + 2 * kb, dv + 2 * kb, idv,
+                                        tbase + PP_SFP + 8 * x + 4 * kb, tbase + PP_SFV + 8 * kb,
+                                        (u > 0 || kb > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&s.o_done[x]);
+                        nP[x]++;
+                    }
+                    if (!ok) break;
+                    tc_commit(&s.kv_empty[st]);  // this tile's P V are issued (the second release)
+                }
+                g0 += I.nu;
+            }
+            tc_commit(&s.drain);
+            pp_drain(&s.drain, 0);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax
-        pp_setmaxnreg_inc<232>();
-        const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
+        pp_setmaxnreg_inc<PP_REG_SM>();
+        const int sw = warp - 4;
+        const int x = sw >> 3;        // 0: tile A, 1: tile B
+        const int h = (sw >> 2) & 1;  // key half: columns 64h..64h+63 of S
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t o_col = tbase + lane_off + PP_O + PP_OW * x;
         const float c2 = p.q_g[0] * p.k_g[0] * p.sm_scale * kLog2e;
+        const float cb = p.sm_scale * kLog2e;              // bf16 scores -> log2 units
+        const float kappa = MIXED ? 2688.0f * p.v_g[1] : 0.0f;  // 2688 / g_V: raw-V units -> accumulator units
         bool ok = true;
-        int k = 0;  // key-tile steps of this tile role so far (all items)
+        int k = 0;   // key-tile steps of this tile so far (all items)
+        int nb = 0;  // this tile's bf16 blocks so far
+        int xp = 0;  // half-row exchanges so far
+        // post this half's value of row r and return the other half's (bounded
+        // wait: both halves count the same exchanges, two slots alternate)
+        auto exchange = [&](float v, float& other) -> bool {
+            s.xch[xp & 1][x][h][r] = v;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.xbar[x][quad]);
+            if (!pp_wait(&s.xbar[x][quad], xp & 1, abort, lim)) return false;
+            other = s.xch[xp & 1][x][h ^ 1][r];
+            xp++;
+            return true;
+        };
         for (int j = 0; ok && j < nrounds; j++) {
             const int i = pp_item_index(j, nitems);
             if (i < 0) continue;
             const PpItem I = pp_item(p, i);
             const int nux = x == 0 ? I.nuA : I.nuB;
-            if (nux == 0) continue;
             const int tq = 2 * I.pair + x;
             const int row = tq * 128 + r;
+            float crow = 0.0f;  // c_i = q_i . mean(K) for this row's bf16 scores
+            if (MIXED && nux > 0 && p.k_mean) {
+                const uint4* qr = reinterpret_cast<const uint4*>(p.q_bf16 + ((size_t)I.bh * p.N + min(row, p.N - 1)) * D);
+                const float* mu = p.k_mean + (size_t)I.bh * D;
+#pragma unroll 4
+                for (int c8 = 0; c8 < D / 8; c8++) {
+                    const uint4 w = __ldg(qr + c8);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        crow = __fmaf_rn(bf16_bits_to_f32(ww[e] & 0xFFFFu), __ldg(mu + 8 * c8 + 2 * e), crow);
+                        crow = __fmaf_rn(bf16_bits_to_f32(ww[e] >> 16), __ldg(mu + 8 * c8 + 2 * e + 1), crow);
+                    }
+                }
+            }
             float m2 = -INFINITY;
+            float lb = 0.0f;  // this half's share of the bf16 row sum (units of 2688 / g_V)
+            PpFlags fl{-64, 0, 0};
             for (int u = 0; u < nux; u++, k++) {
-                if (!pp_wait(&s.s_full[x], k & 1, abort)) {
+                const bool bfx = MIXED && ((pp_flags<MIXED>(fl, p, I, u) >> x) & 1u);
+                if (!pp_wait(&s.s_full[x], k & 1, abort, lim)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                float sv[128];
-#pragma unroll
-                for (int c = 0; c < 4; c++)
-                    tmem_ld32(tbase + lane_off + PP_S + 32 * c, *reinterpret_cast<float(*)[32]>(&sv[32 * c]));
+                float sv[64];
+                tmem_ld32(tbase + lane_off + PP_S + 64 * h, *reinterpret_cast<float(*)[32]>(&sv[0]));
+                tmem_ld32(tbase + lane_off + PP_S + 64 * h + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
                 tmem_wait_ld();
                 reg_fence(sv);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.s_free[x]);
 
-                const int kbase = u * 128;
-                if ((p.causal && u == tq) || (kbase + 128 > p.N)) {
+                const int kbase = u * 128 + 64 * h;
+                float hm;  // this half's max (raw S units for NVFP4, log2 units for bf16)
+                float bmax[4];
+                if (MIXED && bfx) {
+                    hm = -INFINITY;
 #pragma unroll
-                    for (int i2 = 0; i2 < 128; i2++) {
+                    for (int i2 = 0; i2 < 64; i2++) {
                         const int key = kbase + i2;
-                        if (key >= p.N || (p.causal && key > row)) sv[i2] = -INFINITY;
+                        const bool valid = key < p.N && (!p.causal || key <= row);
+                        sv[i2] = valid ? __fsub_rn(sv[i2], crow) * cb : -INFINITY;
+                        hm = fmaxf(hm, sv[i2]);
                     }
-                }
-                float bmax[8];
+                } else {
+                    if ((p.causal && u == tq) || (u * 128 + 128 > p.N)) {
 #pragma unroll
-                for (int blk = 0; blk < 8; blk++) bmax[blk] = pp_max16(&sv[16 * blk]);
-                const float tmax = fmaxf(pp_max3(bmax[0], bmax[1], bmax[2]),
-                                         fmaxf(pp_max3(bmax[3], bmax[4], bmax[5]), fmaxf(bmax[6], bmax[7])));
-                const float m2_new = fmaxf(m2, tmax * c2);
+                        for (int i2 = 0; i2 < 64; i2++) {
+                            const int key = kbase + i2;
+                            if (key >= p.N || (p.causal && key > row)) sv[i2] = -INFINITY;
+                        }
+                    }
+#pragma unroll
+                    for (int blk = 0; blk < 4; blk++) bmax[blk] = pp_max16(&sv[16 * blk]);
+                    hm = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
+                }
+                // the two halves agree on the row max
+                float om;
+                if (!exchange(hm, om)) {
+                    ok = false;
+                    break;
+                }
+                const float tmax = fmaxf(hm, om);
+                const float m2_new = fmaxf(m2, (MIXED && bfx) ? tmax : tmax * c2);
                 const float msub = m2_new == -INFINITY ? 0.0f : m2_new;
                 const float alpha = ex2f(m2 - msub);
                 m2 = m2_new;
-                // block scales first (eight independent chains): E4M3 of (block max of
-                // P * 2688) / 6, and log2 of the scale value from the exponent and a
-                // table of significands
-                const float lm = kLog2_2688 - msub;
-                float bias[8];
-                uint32_t scw0 = 0, scw1 = 0;
+
+                uint32_t codes[8];
+                uint32_t scw = 0;
+                uint32_t pw[MIXED ? 32 : 1];
+                if (MIXED && bfx) {
+                    // P^ = bf16(2^(t - m)) as the method rounds it, then P' = bf16(P^ kappa)
+                    // in the NVFP4 accumulator's units (kappa = 2688 / g_V); the row sum
+                    // of P' is kept per half
+                    float ls = 0.0f;
 #pragma unroll
-                for (int bp = 0; bp < 8; bp += 2) {
-                    const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
-                                                         ex2f(fmaf(bmax[bp + 1], c2, lm)) * (1.0f / 6.0f));
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const int blk = bp + h;
-                        const uint32_t sc = (sc2 >> (8 * h)) & 0xFFu;
-                        bias[blk] = sc ? lm - s.lg2sc[sc] : -INFINITY;
-                        if (blk < 4)
-                            scw0 |= sc << (8 * blk);
-                        else
-                            scw1 |= sc << (8 * (blk - 4));
+                    for (int i2 = 0; i2 < 32; i2++) {
+                        const __nv_bfloat162 ph =
+                            __floats2bfloat162_rn(ex2f(sv[2 * i2] - msub), ex2f(sv[2 * i2 + 1] - msub));
+                        const __nv_bfloat162 pr =
+                            __floats2bfloat162_rn(__low2float(ph) * kappa, __high2float(ph) * kappa);
+                        ls += __low2float(pr);
+                        ls += __high2float(pr);
+                        pw[i2] = *reinterpret_cast<const uint32_t*>(&pr);
                     }
-                }
-                // y = P * 2688 / scale, rounded to E2M1
-                uint32_t codes[16];
+                    lb = lb * alpha + ls;
+                } else {
+                    // block scales first: E4M3 of (block max of P * 2688) / 6, and log2 of
+                    // the scale value from a table
+                    const float lm = kLog2_2688 - msub;
+                    float bias[4];
 #pragma unroll
-                for (int blk = 0; blk < 8; blk++) {
-                    float y[16];
+                    for (int bp = 0; bp < 4; bp += 2) {
+                        const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
+                                                             ex2f(fmaf(bmax[bp + 1], c2, lm)) * (1.0f / 6.0f));
 #pragma unroll
-                    for (int i2 = 0; i2 < 16; i2++) y[i2] = ex2f(fmaf(sv[16 * blk + i2], c2, bias[blk]));
-                    codes[2 * blk] = pack8_e2m1(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-                    codes[2 * blk + 1] = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+                        for (int hh = 0; hh < 2; hh++) {
+                            const int blk = bp + hh;
+                            const uint32_t sc = (sc2 >> (8 * hh)) & 0xFFu;
+                            bias[blk] = sc ? lm - s.lg2sc[sc] : -INFINITY;
+                            scw |= sc << (8 * blk);
+                        }
+                    }
+                    // y = P * 2688 / scale, rounded to E2M1
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; c8++) {
+                        const float* sp = &sv[8 * c8];
+                        const float bs = bias[c8 >> 1];
+                        codes[c8] = pack8_e2m1(ex2f(fmaf(sp[0], c2, bs)), ex2f(fmaf(sp[1], c2, bs)),
+                                               ex2f(fmaf(sp[2], c2, bs)), ex2f(fmaf(sp[3], c2, bs)),
+                                               ex2f(fmaf(sp[4], c2, bs)), ex2f(fmaf(sp[5], c2, bs)),
+                                               ex2f(fmaf(sp[6], c2, bs)), ex2f(fmaf(sp[7], c2, bs)));
+                    }
+                    if (MIXED) lb *= alpha;
                 }
-                // P buffer and O are free once this role's previous P V finished
+                // P buffer and O are free once this tile's previous P V finished
                 // (for u = 0 that is the previous item's last one)
-                if (k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort)) {
+                if (k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint8_t* prow = s.p[x] + (r >> 3) * 512 + (r & 7) * 64;
-#pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    const int cs = c ^ ((r & 7) >> 1);
-                    *reinterpret_cast<uint4*>(prow + cs * 16) =
-                        make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
-                }
-                // P's block scales into TMEM: row r reads (lane r, column base + r / 32)
-                tmem_st1(tbase + lane_off + PP_SFP + 8 * x + quad, __uint_as_float(scw0));
-                tmem_st1(tbase + lane_off + PP_SFP + 8 * x + 4 + quad, __uint_as_float(scw1));
-                if (u > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-                    // rescale this row of O (64 columns per round trip) and l
-                    const uint32_t oa = tbase + lane_off + PP_O + PP_OW * x;
-#pragma unroll
-                    for (int h = 0; h < D / 64; h++) {
-                        float o0[32], o1[32];
-                        tmem_ld32(oa + 64 * h, o0);
-                        tmem_ld32(oa + 64 * h + 32, o1);
-                        tmem_wait_ld();
-                        reg_fence(o0);
-                        reg_fence(o1);
-#pragma unroll
-                        for (int i2 = 0; i2 < 32; i2++) {
-                            o0[i2] *= alpha;
-                            o1[i2] *= alpha;
-                        }
-                        tmem_st32(oa + 64 * h, o0);
-                        tmem_st32(oa + 64 * h + 32, o1);
+                if (MIXED && bfx) {
+                    // the bf16 P buffer is this block's once the bf16 block before it
+                    // (either tile) has finished its P V
+                    if (!pp_wait(&s.pb_grant[x], nb & 1, abort, lim)) {
+                        ok = false;
+                        break;
                     }
-                    const float lv = tmem_ld1_sync(oa + 128);
-                    tmem_st1(oa + 128, lv * alpha);
+                    nb++;
+                    uint8_t* prow = s.pb[h] + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int cc = 0; cc < 8; cc++)
+                        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+                            make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
+                    if (u == 0 && h == 1) tmem_st1(o_col + 128, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
+                } else {
+                    uint8_t* prow = s.p[x] + (r >> 3) * 512 + (r & 7) * 64;
+#pragma unroll
+                    for (int c = 0; c < 2; c++) {
+                        const int cs = (2 * h + c) ^ ((r & 7) >> 1);
+                        *reinterpret_cast<uint4*>(prow + cs * 16) =
+                            make_uint4(codes[4 * c], codes[4 * c + 1], codes[4 * c + 2], codes[4 * c + 3]);
+                    }
+                    // this half's scale word of P: row r reads (lane r, column base + r / 32)
+                    tmem_st1(tbase + lane_off + PP_SFP + 8 * x + 4 * h + quad, __uint_as_float(scw));
+                }
+                if (u > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                    // rescale this half's columns of O (and l, kept by the second half)
+#pragma unroll
+                    for (int c = 0; c < HD; c += 32) {
+                        float o[32];
+                        tmem_ld32(o_col + HD * h + c, o);
+                        tmem_wait_ld();
+                        reg_fence(o);
+#pragma unroll
+                        for (int i2 = 0; i2 < 32; i2++) o[i2] *= alpha;
+                        tmem_st32(o_col + HD * h + c, o);
+                    }
+                    if (h == 1) {
+                        const float lv = tmem_ld1_sync(o_col + 128);
+                        tmem_st1(o_col + 128, lv * alpha);
+                    }
                 }
                 tmem_wait_st();
                 fence_proxy_async();
@@ -458,52 +952,62 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.p_full[x]);
             }
+            if (!ok) break;
+            if (nux == 0) continue;
             // ---- epilogue of this item: out = O / l * g_V (O is reused by the next item
-            // only after this role's next p_full arrival, which follows these loads)
-            if (!ok || !pp_wait(&s.o_done[x], (k - 1) & 1, abort)) {
+            // only after this tile's next p_full arrival, which follows these loads)
+            if (!pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float l = tmem_ld1_sync(tbase + lane_off + PP_O + PP_OW * x + 128);
-            const float scale = p.v_g[0] / l;
+            float den = tmem_ld1_sync(o_col + 128);
+            if (MIXED) {
+                float lo;
+                if (!exchange(lb, lo)) {
+                    ok = false;
+                    break;
+                }
+                den = fmaf(p.v_g[0], lb + lo, den);
+            }
+            const float scale = p.v_g[0] / den;
             {
-                // Stage 32 rows x 16 floats of O per round in this warp's 2 KB of the
-                // tile's P buffer (idle until the next item's first P), 16-byte units
-                // XOR-swizzled by row / 2, then write 64-byte row segments: each store
-                // instruction covers 8 rows.
-                float4* stage = reinterpret_cast<float4*>(s.p[x] + quad * 2048);
+                // Stage 32 rows x 8 floats per round in this warp's 1 KB of the tile's P
+                // buffer (bytes of its own quadrant's rows, which only its partner half
+                // writes, after the next item's first row exchange), 16-byte units
+                // swizzled by row / 4, then
+                // write 32-byte row segments: each store instruction covers 16 rows.
+                float4* stage = reinterpret_cast<float4*>(s.p[x] + quad * 2048 + h * 1024);
                 const int row0 = tq * 128 + quad * 32;
-                float* obase = p.out + ((size_t)I.bh * p.N + row0) * D;
+                float* obase = p.out + ((size_t)I.bh * p.N + row0) * D + HD * h;
 #pragma unroll 1
-                for (int c = 0; c < D / 16; c++) {
-                    uint32_t o[16];
+                for (int c = 0; c < HD / 8; c++) {
+                    uint32_t o[8];
                     asm volatile(
-                        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-                        "%12, %13, %14, %15}, [%16];\n\t"
+                        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
                         "tcgen05.wait::ld.sync.aligned;"
                         : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]),
-                          "=r"(o[7]), "=r"(o[8]), "=r"(o[9]), "=r"(o[10]), "=r"(o[11]), "=r"(o[12]), "=r"(o[13]),
-                          "=r"(o[14]), "=r"(o[15])
-                        : "r"(tbase + lane_off + PP_O + PP_OW * x + 16 * c)
+                          "=r"(o[7])
+                        : "r"(o_col + HD * h + 8 * c)
                         : "memory");
 #pragma unroll
-                    for (int j2 = 0; j2 < 4; j2++)
-                        stage[lane * 4 + (j2 ^ ((lane >> 1) & 3))] =
+                    for (int j2 = 0; j2 < 2; j2++)
+                        stage[2 * lane + (j2 ^ ((lane >> 2) & 1))] =
                             make_float4(__uint_as_float(o[4 * j2]) * scale, __uint_as_float(o[4 * j2 + 1]) * scale,
                                         __uint_as_float(o[4 * j2 + 2]) * scale, __uint_as_float(o[4 * j2 + 3]) * scale);
                     __syncwarp();
 #pragma unroll
-                    for (int i2 = 0; i2 < 4; i2++) {
-                        const int rr = 8 * i2 + (lane >> 2), jj = lane & 3;
+                    for (int i2 = 0; i2 < 2; i2++) {
+                        const int rr = 16 * i2 + (lane >> 1), uu = lane & 1;
                         if (row0 + rr < p.N)
-                            *reinterpret_cast<float4*>(obase + (size_t)rr * D + 16 * c + 4 * jj) =
-                                stage[rr * 4 + (jj ^ ((rr >> 1) & 3))];
+                            *reinterpret_cast<float4*>(obase + (size_t)rr * D + 8 * c + 4 * uu) =
+                                stage[2 * rr + (uu ^ ((rr >> 2) & 1))];
                     }
                     __syncwarp();
                 }
             }
-            if (p.lse && row < p.N) p.lse[(size_t)I.bh * p.N + row] = m2 * kLn2 + logf(l * (1.0f / 2688.0f));
+            if (p.lse && h == 0 && row < p.N)
+                p.lse[(size_t)I.bh * p.N + row] = m2 * kLn2 + logf(den * (1.0f / 2688.0f));
             tc_fence_before();
         }
     }

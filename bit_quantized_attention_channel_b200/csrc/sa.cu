@@ -51,6 +51,61 @@ int sm_count()
     return n;
 }
 
+// One value per device (kernel attributes and occupancy are per device:
+// cudaFuncSetAttribute and the occupancy query act on the current one).
+// Host threads may race on a device's first use; they store the same value.
+struct PerDevice {
+    std::atomic<int> v[64];
+};
+
+int current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev >= 0 && dev < 64 ? dev : -1;
+}
+
+// Run `set` (returning a positive value, or <= 0 on failure) once per device
+// and return the cached value; 0 on failure.
+template <typename F>
+int once_per_device(PerDevice& pd, F&& set)
+{
+    const int dev = current_device();
+    if (dev < 0) return 0;
+    int v = pd.v[dev].load(std::memory_order_acquire);
+    if (v > 0) return v;
+    v = set();
+    if (v <= 0) return 0;
+    pd.v[dev].store(v, std::memory_order_release);
+    return v;
+}
+
+// Opt a kernel into `smem` bytes of dynamic shared memory on the current
+// device (once per device); false on failure.
+template <typename K>
+bool allow_smem(PerDevice& pd, K kernel, int smem)
+{
+    return once_per_device(pd, [&] {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1 : 0;
+    }) > 0;
+}
+
+// Limit of every pipeline wait of the attention kernel, in SM clock cycles
+// (0: the library default, about 2 s at the B200 clock).
+std::atomic<long long> g_wait_cycles{0};
+
+// The attention kernel moves registers between its warps with setmaxnreg;
+// an increase waits until the CTA's launch allocation (threads x registers
+// per thread, fixed by the compiler) has room, so a split larger than that
+// allocation would never proceed.  Refuse to launch such a build.
+template <typename K>
+bool pp_regs_fit(K kernel)
+{
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return false;
+    return (long)fa.numRegs * kPpThreads >= 128L * PP_REG_CTL + 512L * PP_REG_SM;
+}
+
 // 3-D byte tensor {d0 (contiguous), d1, d2}; box {b0, b1, 1}.
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                  uint32_t b1, CUtensorMapSwizzle swz)
@@ -108,6 +163,8 @@ const char* sa_status_string(sa_status s)
     }
     return "SA_ERR_UNKNOWN";
 }
+
+void sa_set_wait_cycles(long long cycles) { g_wait_cycles.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed); }
 
 sa_status sa_device_status(cudaStream_t stream, int reset)
 {
@@ -329,17 +386,18 @@ sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v
 #define SA_PQ(DD, SS, SM)                                                                                      \
     do {                                                                                                       \
         const int smem = (int)sizeof(PqSmem<DD>);                                                              \
-        /* set on the first call, outside any stream capture; racing first calls store the same value */     \
-        static std::atomic<int> per_sm_cache{0};                                                               \
-        int per_sm = per_sm_cache.load(std::memory_order_acquire);                                             \
-        if (!per_sm) {                                                                                         \
+        /* set on a device's first call, outside any stream capture */                                      \
+        static PerDevice per_sm_cache;                                                                         \
+        const int per_sm = once_per_device(per_sm_cache, [&] {                                                 \
+            int n = 0;                                                                                         \
             if (cudaFuncSetAttribute(prepass_quant_kernel<DD, SS, SM>,                                         \
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||      \
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prepass_quant_kernel<DD, SS, SM>, 2 * DD, \
-                                                              smem) != cudaSuccess || per_sm < 1)              \
-                return SA_ERR_CUDA;                                                                            \
-            per_sm_cache.store(per_sm, std::memory_order_release);                                             \
-        }                                                                                                      \
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, prepass_quant_kernel<DD, SS, SM>, 2 * DD,    \
+                                                              smem) != cudaSuccess)                            \
+                return 0;                                                                                      \
+            return n;                                                                                          \
+        });                                                                                                    \
+        if (per_sm < 1) return SA_ERR_CUDA;                                                                    \
         const unsigned gq = (unsigned)std::min<long>(3L * BH * T, (long)per_sm * sm_count());                  \
         prepass_quant_kernel<DD, SS, SM><<<gq, 2 * DD, smem, stream>>>(p);                                     \
     } while (0)
@@ -458,43 +516,28 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     p.mask = mask_dev;
     p.q_bf16 = (const uint16_t*)q_bf16_dev;
     p.k_mean = k_mean_dev;
-    dim3 grid(p.T, H, B);
+    const long long wc = g_wait_cycles.load(std::memory_order_relaxed);
+    p.wait_cycles = wc > 0 ? wc : SA_WAIT_CYCLES;
+    const long nitems = (long)B * H * ((p.T + 1) / 2);
+    const int nsm = sm_count();
+    if (nsm <= 0) return SA_ERR_CUDA;
+    const unsigned grid = (unsigned)(nitems < nsm ? nitems : nsm);  // persistent: one CTA per SM
 #define SA_ATTN_LAUNCH(DD, MX)                                                                              \
     do {                                                                                                    \
-        const int smem = MX ? (int)(((sizeof(AttnSmem<DD>) + 1023) & ~(size_t)1023) + sizeof(MixedSmem<DD>) + \
-                                    1024)                                                                   \
-                            : 116 * 1024; /* one CTA per SM: the CTA owns all 512 TMEM columns */          \
-        static std::atomic<int> attr_done{0}; /* set once, outside any stream capture */                \
-        if (!attr_done.load(std::memory_order_acquire)) {                                                   \
-            if (cudaFuncSetAttribute(attn_fwd_kernel<DD, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
-                                     smem) != cudaSuccess)                                                  \
-                return SA_ERR_CUDA;                                                                         \
-            attr_done.store(1, std::memory_order_release);                                                  \
-        }                                                                                                   \
-        attn_fwd_kernel<DD, MX><<<grid, 128, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);                 \
-    } while (0)
-#define SA_ATTN_PP_LAUNCH(DD)                                                                               \
-    do {                                                                                                    \
-        const int smem = (int)sizeof(PpSmem<DD>) + 1024;                                                    \
-        static std::atomic<int> attr_done{0};                                                               \
-        if (!attr_done.load(std::memory_order_acquire)) {                                                   \
-            if (cudaFuncSetAttribute(attn_fwd_pp_kernel<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                     smem) != cudaSuccess)                                                  \
-                return SA_ERR_CUDA;                                                                         \
-            attr_done.store(1, std::memory_order_release);                                                  \
-        }                                                                                                   \
-        const long nitems = (long)B * H * ((p.T + 1) / 2);                                                \
-        const int nsm = sm_count();                                                                         \
-        if (nsm <= 0) return SA_ERR_CUDA;                                                                   \
-        attn_fwd_pp_kernel<DD><<<(unsigned)(nitems < nsm ? nitems : nsm), kPpThreads, smem, stream>>>(tq, tk, tv, p); \
+        const int smem = (int)sizeof(PpSmem<DD, MX>) + 1024;                                                \
+        static PerDevice attr; /* set on a device's first call, outside any stream capture */              \
+        if (!allow_smem(attr, attn_fwd_pp_kernel<DD, MX>, smem)) return SA_ERR_CUDA;                        \
+        static PerDevice regs_ok; /* the kernel's register split must fit its launch allocation */         \
+        if (once_per_device(regs_ok, [] { return pp_regs_fit(attn_fwd_pp_kernel<DD, MX>) ? 1 : 0; }) <= 0)  \
+            return SA_ERR_UNSUPPORTED;                                                                      \
+        attn_fwd_pp_kernel<DD, MX><<<grid, kPpThreads, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);       \
     } while (0)
     if (D == 128) {
-        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_PP_LAUNCH(128);
+        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_LAUNCH(128, false);
     } else {
-        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_PP_LAUNCH(64);
+        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_LAUNCH(64, false);
     }
 #undef SA_ATTN_LAUNCH
-#undef SA_ATTN_PP_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
 }
@@ -556,23 +599,13 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
     dim3 grid(nsplit, Hkv, B);
     if (D == 128) {
         const int smem = (int)sizeof(DecSmem<128>) + 1024;
-        static std::atomic<int> attr_done{0};
-        if (!attr_done.load(std::memory_order_acquire)) {
-            if (cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess)
-                return SA_ERR_CUDA;
-            attr_done.store(1, std::memory_order_release);
-        }
+        static PerDevice attr;
+        if (!allow_smem(attr, decode_kernel<128>, smem)) return SA_ERR_CUDA;
         decode_kernel<128><<<grid, 128, smem, stream>>>(tk, tv, p);
     } else {
         const int smem = (int)sizeof(DecSmem<64>) + 1024;
-        static std::atomic<int> attr_done{0};
-        if (!attr_done.load(std::memory_order_acquire)) {
-            if (cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-                cudaSuccess)
-                return SA_ERR_CUDA;
-            attr_done.store(1, std::memory_order_release);
-        }
+        static PerDevice attr;
+        if (!allow_smem(attr, decode_kernel<64>, smem)) return SA_ERR_CUDA;
         decode_kernel<64><<<grid, 128, smem, stream>>>(tk, tv, p);
     }
     SA_CHECK_LAUNCH();

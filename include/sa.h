@@ -90,6 +90,16 @@ const char* sa_status_string(sa_status s);
  * earlier calls (SA_OK if none) and clears it when `reset` != 0. */
 sa_status sa_device_status(cudaStream_t stream, int reset);
 
+/* Limit, in SM clock cycles, of every pipeline wait inside sa_attn_fwd's
+ * kernel, for the calls made after it (process-wide); cycles <= 0 restores
+ * the default (about 2 s at the B200 clock).  A wait that reaches the limit
+ * records SA_ERR_TIMEOUT, every warp of the CTA unwinds, copies and
+ * tensor-core work already issued are waited for, and the kernel returns;
+ * the output of that call is then undefined, and later calls run normally.
+ * A short limit (hundreds of cycles, below one copy's latency) makes a call
+ * give up on purpose, which is how the timeout path is tested. */
+void sa_set_wait_cycles(long long cycles);
+
 /* Byte sizes of the NVFP4 code and scale buffers of one tensor. */
 size_t sa_codes_bytes(int B, int H, int N, int D, sa_role role);
 size_t sa_scales_bytes(int B, int H, int N, int D, sa_role role);

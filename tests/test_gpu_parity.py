@@ -341,7 +341,10 @@ def test_mixed_attention_matches_oracle(mask_kind, causal, N, D):
     qo, ko, vo = orc.quantize(q, "q"), orc.quantize(k, "k"), orc.quantize(v, "v")
     ref, lse_ref = orc.attention(qo, ko, vo, causal, mask=mask, q_bf16=q, k_bf16=k, v_bf16=v, want_lse=True)
     check_close(og, ref, f"mixed {mask_kind} causal={causal} N={N} D={D}")
-    assert np.max(np.abs(lg - lse_ref)) < 1e-3
+    # a bf16 block's P is rounded to bf16 as the method states, then scaled into
+    # the NVFP4 accumulator's units and rounded again: the denominator can
+    # differ by up to 2^-8 relative where bf16 blocks dominate a row
+    assert np.max(np.abs(lg - lse_ref)) < 4e-3
     # with no block selected the mixed kernel computes the NVFP4 result
     if mask_kind == "select":
         og0, _ = run_mixed(q, k, v, causal, np.zeros_like(mask))
@@ -368,3 +371,24 @@ def test_mixed_full_size_sampled():
     e4 = np.linalg.norm(fp4 - ex)
     emx = np.linalg.norm(ref - ex)
     print(f"  FP4->exact gap recovered by 5% bf16 blocks: {100 * (1 - emx / e4):.1f}%")
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_wait_limit_gives_up_cleanly_and_the_next_call_is_normal():
+    """A wait limit far below one copy's latency makes the attention kernel's
+    first pipeline wait give up: the call reports SA_ERR_TIMEOUT through the
+    status word (every warp unwinds, issued copies and MMAs are drained), and
+    with the default limit restored the next call runs and matches the oracle.
+    Nothing is broken on purpose: every arrive still happens."""
+    q, k, v = inputs("tiny")
+    qg, kg, vg = (gpu_quant(x, r) for x, r in ((q, "q"), (k, "k"), (v, "v")))
+    try:
+        sa.sa_set_wait_cycles(200)
+        sa.sa_attn_fwd(qg, kg, vg, False)
+        assert sa.sa_device_status(reset=True) == 6  # SA_ERR_TIMEOUT
+    finally:
+        sa.sa_set_wait_cycles(0)
+    out = sa.sa_attn_fwd(qg, kg, vg, False)
+    status_ok()
+    qo, ko, vo = orc.quantize(q, "q"), orc.quantize(k, "k"), orc.quantize(v, "v")
+    check_close(out.cpu().numpy(), orc.attention(qo, ko, vo, False), "attention after a timed-out call")

@@ -79,3 +79,23 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = argparse.Namespace(steps=1, warmup=3, mode="max")
     assert bench.run_reference(args, wl.WORKLOADS["llm"], rank=1, world=2) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_reports_the_steps_it_ran(capsys):
+    """The reference arm runs W untimed and K timed oracle samples; its line
+    carries K and W and a per-step time that the run's own wall time covers."""
+    import json
+    import time
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from bit_quantized_attention_channel_b200 import workloads as wl
+
+    args = argparse.Namespace(steps=2, warmup=3, mode="max")
+    t0 = time.perf_counter()
+    bench.run_reference(args, wl.WORKLOADS["tiny"], rank=0, world=1)
+    wall = time.perf_counter() - t0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3
+    assert 0 < line["ms_per_step"] * line["steps"] / 1e3 <= wall
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
