@@ -70,6 +70,13 @@ struct PpSmem {
     alignas(16) uint8_t qsf[QB][2][D / 64 * 512];
     uint8_t ksf[S][D / 64 * 512];
     uint8_t vsf[S][2 * 512];
+    // Key tiles holding a bf16 block, in schedule order: {item count, key tile,
+    // flags (bit x: query tile x), b*H + h | pair << 16}.  The producer pushes
+    // an entry just before it loads that tile into the ring, so every role
+    // that has waited for the tile finds it; at most S such tiles are in
+    // flight, far below the 16 slots.
+    int4 bfq[16];
+    int bfq_n;                // entries pushed
     float lg2sc[128];         // log2 of each nonzero E4M3 scale value
     float xch[2][2][2][128];  // half-row exchange: [use parity][tile][half][row]
     uint64_t q_full[QB];      // Q tiles and scale atoms landed
@@ -189,15 +196,6 @@ SA_DEV PpItem pp_item(const AttnParams& p, int i)
     return it;
 }
 
-// Is the block (query tile x of the item, key tile u) a bf16 block?
-template <bool MIXED>
-SA_DEV bool pp_bf16(const AttnParams& p, const PpItem& I, int x, int u)
-{
-    if (!MIXED) return false;
-    if (u >= (x ? I.nuB : I.nuA)) return false;
-    return __ldg(p.mask + ((size_t)I.bh * p.T + 2 * I.pair + x) * p.T + u) != 0;
-}
-
 // bf16 flags of key tiles [base, base + 32) of an item's two query tiles, read
 // from the mask once per 32 tiles instead of per tile.
 struct PpFlags {
@@ -254,6 +252,25 @@ SA_DEV uint32_t pp_flags(PpFlags& f, const AttnParams& p, const PpItem& I, int u
     return ((f.a >> i) & 1u) | (((f.b >> i) & 1u) << 1);
 }
 
+// bf16 flags of key tile u of the item counted `it` (bit x: query tile x),
+// read from the queue the producer fills; `qi` is the caller's read position
+// (entries are in schedule order, so it only moves forward).
+template <bool MIXED, typename Q>
+SA_DEV uint32_t pp_bf16_flags(const Q& s, int& qi, int it, int u)
+{
+    if (!MIXED) return 0;
+    const int n = *reinterpret_cast<const volatile int*>(&s.bfq_n);
+    const long long key = ((long long)it << 32) | (unsigned)u;
+    while (qi < n) {
+        const int4 e = s.bfq[qi & 15];
+        const long long ek = ((long long)e.x << 32) | (unsigned)e.y;
+        if (ek > key) return 0;
+        qi++;
+        if (ek == key) return (uint32_t)e.z;
+    }
+    return 0;
+}
+
 // Position of the producer's walk over this CTA's items and their key tiles.
 struct PpCursor {
     int j;   // round
@@ -286,66 +303,57 @@ SA_DEV void pp_cursor_next_item(PpCursor& c, const AttnParams& p, int nitems, in
     pp_cursor_seek_item(c, p, nitems, nrounds);
 }
 
-// Could any of the 16 key tiles u0..u0+15 of the item hold a bf16 block?  (A
-// cheap skip for the long runs of NVFP4 tiles: one 16-byte load per mask row
-// when the rows are 16-byte aligned; false means certainly not.)
-template <bool MIXED>
-SA_DEV bool pp_maybe_bf16_x16(const AttnParams& p, const PpItem& I, int u0)
+// The P of a bf16 block for one half row, eight keys at a time from S (which
+// the block still holds): t = (S - c_i) sm_scale log2(e) (masked keys none),
+// P^ = bf16(2^(t - m)) as the method rounds it, then P' = bf16(P^ kappa) in
+// the NVFP4 accumulator's units (kappa = 2688 / g_V), written to the bf16 P
+// row (128-byte swizzle).  Returns the sum of P'.  Kept out of line: bf16
+// blocks are few and the softmax loop stays compact.
+__device__ __noinline__ float pp_bf16_p_row(uint8_t* prow, uint32_t s_col, int swz, int kbase, bool edge, int N,
+                                            bool causal, int row, float crow, float cb, float msub, float kappa)
 {
-    if (!MIXED) return false;
-    if ((p.T & 15) || u0 + 16 > p.T) return true;
-    const uint8_t* row = p.mask + ((size_t)I.bh * p.T + 2 * I.pair) * p.T + u0;
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(row));
-    uint32_t any = a.x | a.y | a.z | a.w;
-    if (I.hasB) {
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(row + p.T));
-        any |= b.x | b.y | b.z | b.w;
+    float ls = 0.0f;
+#pragma unroll 1
+    for (int cc = 0; cc < 8; cc++) {
+        float sc[8];
+        tmem_ld8_sync(s_col + 8 * cc, sc);
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            float t2[2];
+#pragma unroll
+            for (int j2 = 0; j2 < 2; j2++) {
+                const int key = kbase + 8 * cc + 2 * e + j2;
+                const bool valid = !edge || (key < N && (!causal || key <= row));
+                t2[j2] = valid ? ex2f(__fsub_rn(sc[2 * e + j2], crow) * cb - msub) : 0.0f;
+            }
+            const __nv_bfloat162 ph = __floats2bfloat162_rn(t2[0], t2[1]);
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(__low2float(ph) * kappa, __high2float(ph) * kappa);
+            ls += __low2float(pr);
+            ls += __high2float(pr);
+            w4[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        *reinterpret_cast<uint4*>(prow + ((cc ^ swz) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
-    return any != 0;
+    return ls;
 }
 
-// Advance to the first key tile at or after c.u (crossing items) that holds a
-// bf16 block of either query tile.  At most `budget` probes per call: returns
-// 1 (found), 0 (not yet: call again) or -1 (past the end).
-template <bool MIXED>
-SA_DEV int pp_next_bf16_tile(PpCursor& c, const AttnParams& p, int nitems, int nrounds, int budget)
+// c_i = q_i . mean(K) for one query row (bf16 q, FP32 means), an FP32 fma
+// chain over the channels in order.  Once per item; kept out of line.
+__device__ __noinline__ float pp_row_offset(const uint16_t* qrow, const float* mu, int d)
 {
-    while (c.i >= 0) {
-        while (c.u < c.I.nu) {
-            if (budget-- <= 0) return 0;
-            if ((c.u & 15) == 0 && !pp_maybe_bf16_x16<MIXED>(p, c.I, c.u)) {
-                c.u += 16;
-                continue;
-            }
-            if (pp_bf16<MIXED>(p, c.I, 0, c.u) || pp_bf16<MIXED>(p, c.I, 1, c.u)) return 1;
-            c.u++;
+    float c = 0.0f;
+#pragma unroll 1
+    for (int c8 = 0; c8 < d / 8; c8++) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(qrow) + c8);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            c = __fmaf_rn(bf16_bits_to_f32(ww[e] & 0xFFFFu), __ldg(mu + 8 * c8 + 2 * e), c);
+            c = __fmaf_rn(bf16_bits_to_f32(ww[e] >> 16), __ldg(mu + 8 * c8 + 2 * e + 1), c);
         }
-        pp_cursor_next_item(c, p, nitems, nrounds);
     }
-    return -1;
-}
-
-// Advance to the first bf16 block (x, u) at or after (c.u, c.x) in the order
-// u ascending, then x (the issue order of Q K^T and of P V); budget and
-// return value as pp_next_bf16_tile.
-template <bool MIXED>
-SA_DEV int pp_next_bf16_block(PpCursor& c, const AttnParams& p, int nitems, int nrounds, int budget)
-{
-    while (c.i >= 0) {
-        while (c.u < c.I.nu) {
-            if (budget-- <= 0) return 0;
-            if (c.x == 0 && (c.u & 15) == 0 && !pp_maybe_bf16_x16<MIXED>(p, c.I, c.u)) {
-                c.u += 16;
-                continue;
-            }
-            for (; c.x < 2; c.x++)
-                if (pp_bf16<MIXED>(p, c.I, c.x, c.u)) return 1;
-            c.x = 0;
-            c.u++;
-        }
-        pp_cursor_next_item(c, p, nitems, nrounds);
-    }
-    return -1;
+    return c;
 }
 
 template <int D, bool MIXED>
@@ -377,6 +385,8 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
     }
     if (tid == 0) {
         s.abort = 0;
+        s.bfq_n = 0;
+        for (int i = 0; i < 16; i++) s.bfq[i] = make_int4(-1, -1, 0, 0);
         for (int i = 0; i < QB; i++) {
             mbar_init(&s.q_full[i], 1);
             mbar_init(&s.q_empty[i], 1);
@@ -457,19 +467,14 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             cr = cf;
             int rg = 0;  // K/V tiles loaded so far (ring position)
             int nqf[QB] = {};  // Q loads per Q buffer
-            // bf16 streams: state 1 = at the next bf16 tile (block), 0 = still
-            // scanning the mask (a few probes per poll), -1 = past the end
-            PpCursor ck{}, cv{}, cq{};
-            int kst = -1, vst = -1, qst = -1;
+            // bf16 streams read the queue the ring fills: raw K and raw V tiles in
+            // queue order, raw Q tiles per bf16 block (query tile x of an entry)
+            int kq = 0, vq = 0, qq = 0, qx = 0;        // queue positions of the three streams
             int nk = 0, nv = 0, nrl = 0, qhold = -1;  // raw K, V tiles and raw Q reloads issued
-            if (MIXED) {
-                ck = cf;
-                cv = cf;
-                cq = cf;
-                kst = vst = qst = 0;
-            }
+            PpFlags fr{-64, 0, 0};                    // the ring's view of the mask
+            int fr_it = -1;
             long long t_last = clock64();
-            while (cf.i >= 0 || cr.i >= 0 || kst >= 0 || vst >= 0 || qst >= 0) {
+            while (cf.i >= 0 || cr.i >= 0 || (MIXED && (kq < s.bfq_n || vq < s.bfq_n || qq < s.bfq_n))) {
                 bool prog = false;
                 if (cf.i >= 0) {
                     const PpItem& I = cf.I;
@@ -493,6 +498,19 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     const PpItem& I = cr.I;
                     const int st = rg % S, u = cr.u;
                     if (rg < S || mbar_test(&s.kv_empty[st], ((rg / S) & 1) ^ 1)) {
+                        if (MIXED) {
+                            // publish the tile's bf16 flags before its data can be waited for
+                            if (fr_it != cr.it) {
+                                fr = PpFlags{-64, 0, 0};
+                                fr_it = cr.it;
+                            }
+                            const uint32_t f = pp_flags<MIXED>(fr, p, I, u);
+                            if (f) {
+                                const int n = s.bfq_n;
+                                s.bfq[n & 15] = make_int4(cr.it, u, (int)f, I.bh | (I.pair << 16));
+                                *reinterpret_cast<volatile int*>(&s.bfq_n) = n + 1;
+                            }
+                        }
                         const int nk2 = min(128, p.N - u * 128);
                         const int kblocks = nk2 > 64 ? 2 : 1;
                         mbar_expect_tx(&s.kv_full[st], 128 * D / 2 + KB * 512 + D * 64 + kblocks * 512);
@@ -508,52 +526,57 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     }
                 }
                 if (MIXED) {
-                    constexpr int kProbe = 8;  // mask probes per stream and poll
-                    if (kst == 0 && (kst = pp_next_bf16_tile<MIXED>(ck, p, nitems, nrounds, kProbe)) >= 0) prog = true;
-                    if (vst == 0 && (vst = pp_next_bf16_tile<MIXED>(cv, p, nitems, nrounds, kProbe)) >= 0) prog = true;
-                    if (qst == 0 && (qst = pp_next_bf16_block<MIXED>(cq, p, nitems, nrounds, kProbe)) >= 0) prog = true;
-                    // raw K of bf16 key tile nk: the previous one's Q K^T have completed
-                    if (kst == 1 && (nk == 0 || mbar_test(&s.kb_empty, (nk - 1) & 1))) {
+                    const int n = s.bfq_n;
+                    // raw K of the next queued tile: the previous one's Q K^T have completed
+                    if (kq < n && (nk == 0 || mbar_test(&s.kb_empty, (nk - 1) & 1))) {
+                        const int4 e = s.bfq[kq & 15];
                         mbar_expect_tx(&s.kb_full, 128 * D * 2);
                         for (int r = 0; r < D / 64; r++)
-                            tma_load_3d(s.kb[r], &tm_kb, &s.kb_full, 64 * r, ck.u * 128, ck.I.bh);
+                            tma_load_3d(s.kb[r], &tm_kb, &s.kb_full, 64 * r, e.y * 128, e.w & 0xFFFF);
                         nk++;
-                        ck.u++;
-                        kst = 0;
+                        kq++;
                         prog = true;
                     }
-                    // raw V of bf16 key tile nv: the previous one's P V have completed
-                    if (vst == 1 && (nv == 0 || mbar_test(&s.vb_empty, (nv - 1) & 1))) {
+                    // raw V of the next queued tile: the previous one's P V have completed
+                    if (vq < n && (nv == 0 || mbar_test(&s.vb_empty, (nv - 1) & 1))) {
+                        const int4 e = s.bfq[vq & 15];
                         mbar_expect_tx(&s.vb_full, 128 * D * 2);
                         for (int r = 0; r < D / 64; r++)
-                            tma_load_3d(s.vb[r], &tm_vb, &s.vb_full, 64 * r, cv.u * 128, cv.I.bh);
+                            tma_load_3d(s.vb[r], &tm_vb, &s.vb_full, 64 * r, e.y * 128, e.w & 0xFFFF);
                         nv++;
-                        cv.u++;
-                        vst = 0;
+                        vq++;
                         prog = true;
                     }
                     // raw Q for the next bf16 block: reload when it is another query
                     // tile's, once the issuer has released the buffer (one qb_empty
                     // phase per reload)
-                    if (qst == 1) {
-                        const int want = cq.it * 2 + cq.x;
-                        bool go = want == qhold;
-                        if (!go && (nrl == 0 || mbar_test(&s.qb_empty, (nrl - 1) & 1))) {
-                            mbar_expect_tx(&s.qb_full, 128 * D * 2);
-                            for (int r = 0; r < D / 64; r++)
-                                tma_load_3d(s.qb[r], &tm_qb, &s.qb_full, 64 * r, (2 * cq.I.pair + cq.x) * 128,
-                                            cq.I.bh);
-                            qhold = want;
-                            nrl++;
-                            go = true;
-                        }
-                        if (go) {
-                            if (++cq.x == 2) {
-                                cq.x = 0;
-                                cq.u++;
+                    if (qq < n) {
+                        const int4 e = s.bfq[qq & 15];
+                        if (!((e.z >> qx) & 1)) {
+                            if (++qx == 2) {
+                                qx = 0;
+                                qq++;
                             }
-                            qst = 0;
                             prog = true;
+                        } else {
+                            const int want = e.x * 2 + qx;
+                            bool go = want == qhold;
+                            if (!go && (nrl == 0 || mbar_test(&s.qb_empty, (nrl - 1) & 1))) {
+                                mbar_expect_tx(&s.qb_full, 128 * D * 2);
+                                for (int r = 0; r < D / 64; r++)
+                                    tma_load_3d(s.qb[r], &tm_qb, &s.qb_full, 64 * r, (2 * (e.w >> 16) + qx) * 128,
+                                                e.w & 0xFFFF);
+                                qhold = want;
+                                nrl++;
+                                go = true;
+                            }
+                            if (go) {
+                                if (++qx == 2) {
+                                    qx = 0;
+                                    qq++;
+                                }
+                                prog = true;
+                            }
                         }
                     }
                 }
@@ -566,6 +589,10 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                         sa_raise(SA_ERR_TIMEOUT);
                         break;
                     }
+                    // nothing to do yet: back off instead of taking issue slots from
+                    // the softmax warps of this SM sub-partition (the ring holds
+                    // several key tiles of slack)
+                    __nanosleep(128);
                 }
             }
             // every copy issued has landed before the CTA releases its shared memory
@@ -597,6 +624,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             int nS[2] = {0, 0};
             int it = 0;
             int bk = 0, bq = 0, qhold = -1;  // bf16: raw K tiles and raw Q loads used so far
+            int bq_pos = 0;                  // read position in the bf16 tile queue
             for (int j = 0; ok && j < nrounds; j++) {
                 const int i = pp_item_index(j, nitems);
                 if (i < 0) continue;
@@ -607,12 +635,15 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 for (int x = 0; x < (I.hasB ? 2 : 1); x++)
                     for (int kb = 0; kb < KB; kb++)
                         tc_cp_sf(tbase + PP_SFQ + 8 * x + 4 * kb, smem_u32(s.qsf[qs][x] + 512 * kb));
-                PpFlags fl{-64, 0, 0};
                 for (int u = 0; ok && u < I.nu; u++) {
                     const int gt = g0 + u, st = gt % S;
-                    const uint32_t f = pp_flags<MIXED>(fl, p, I, u);
                     if (!(ok = pp_wait(&s.kv_full[st], (gt / S) & 1, abort, lim))) break;
-                    bool sfk = false;
+                    const uint32_t f = pp_bf16_flags<MIXED>(s, bq_pos, it, u);
+                    // K scale atoms of this tile, queued behind the previous tile's Q K^T
+                    // (the tensor pipe runs them in issue order) while S is still busy
+                    tc_fence_after();
+                    for (int kb = 0; kb < KB; kb++)
+                        tc_cp_sf(tbase + PP_SFK + 4 * kb, smem_u32(s.ksf[st] + 512 * kb));
                     for (int x = 0; x < 2; x++) {
                         if (u >= (x ? I.nuB : I.nuA)) continue;
                         if (last_x >= 0 && !(ok = pp_wait(&s.s_free[last_x], last_idx & 1, abort, lim))) break;
@@ -630,20 +661,18 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                                 qhold = want;
                             }
                             tc_fence_after();
-                            for (int ks = 0; ks < D / 16; ks++)
-                                mma_bf16(tbase + PP_S, make_sdesc(smem_u32(s.qb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                                         make_sdesc(smem_u32(s.kb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                                         idesc_bf16(128, 128, 0), ks > 0);
+                            const uint64_t dqb = make_sdesc(smem_u32(&s.qb[0][0]), 1024, 16, 2);
+                            const uint64_t dkb = make_sdesc(smem_u32(&s.kb[0][0]), 1024, 16, 2);
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ks++) {
+                                const uint64_t o = (uint64_t)(((ks >> 2) * 16384 + 32 * (ks & 3)) >> 4);
+                                mma_bf16(tbase + PP_S, dqb + o, dkb + o, idesc_bf16(128, 128, 0), ks > 0);
+                            }
                             if (x == 1 || !(f & 2)) {  // last bf16 Q K^T of this key tile
                                 tc_commit(&s.kb_empty);
                                 bk++;
                             }
                         } else {
-                            if (!sfk) {
-                                for (int kb = 0; kb < KB; kb++)
-                                    tc_cp_sf(tbase + PP_SFK + 4 * kb, smem_u32(s.ksf[st] + 512 * kb));
-                                sfk = true;
-                            }
                             const uint64_t dq = dq0 + (uint64_t)(((qs * 2 + x) * (128 * D / 2)) >> 4);
                             const uint64_t dk = dk0 + (uint64_t)((st * (128 * D / 2)) >> 4);
 #pragma unroll
@@ -679,23 +708,17 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             int g0 = 0;
             int nP[2] = {0, 0};
             int bv = 0;  // bf16: raw V tiles used so far
-            // the next bf16 block after the one being issued (hands the bf16 P buffer on)
-            PpCursor nx{};
-            int nx_st = -1;
-            if (MIXED) {
-                pp_cursor_seek_item(nx, p, nitems, nrounds);
-                nx_st = pp_next_bf16_block<MIXED>(nx, p, nitems, nrounds, 1 << 30);
-                if (nx_st == 1) mbar_arrive(&s.pb_grant[nx.x]);  // the first bf16 block may write P at once
-            }
+            bool first_bf = true;  // no bf16 block handed the bf16 P buffer yet
+            int bq_pos = 0;        // read position in the bf16 tile queue
+            int it = 0;
             for (int j = 0; ok && j < nrounds; j++) {
                 const int i = pp_item_index(j, nitems);
                 if (i < 0) continue;
                 const PpItem I = pp_item(p, i);
-                PpFlags fl{-64, 0, 0};
                 for (int u = 0; ok && u < I.nu; u++) {
                     const int gt = g0 + u, st = gt % S;
-                    const uint32_t f = pp_flags<MIXED>(fl, p, I, u);
                     if (!(ok = pp_wait(&s.kv_full[st], (gt / S) & 1, abort, lim))) break;
+                    const uint32_t f = pp_bf16_flags<MIXED>(s, bq_pos, it, u);
                     tc_fence_after();
                     // V scale atoms of key tile u (the P V of the tile before was issued earlier)
                     const int nk = min(128, p.N - u * 128);
@@ -704,23 +727,29 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                         tc_cp_sf(tbase + PP_SFV + 8 * kb, smem_u32(s.vsf[st] + 512 * kb));
                     for (int x = 0; x < 2; x++) {
                         if (u >= (x ? I.nuB : I.nuA)) continue;
+                        if (MIXED && ((f >> x) & 1)) {
+                            // this bf16 block may write the shared bf16 P buffer once the
+                            // P V issued so far (the previous bf16 block's among them)
+                            // have completed
+                            if (first_bf)
+                                mbar_arrive(&s.pb_grant[x]);
+                            else
+                                tc_commit(&s.pb_grant[x]);
+                            first_bf = false;
+                        }
                         if (!(ok = pp_wait(&s.p_full[x], nP[x] & 1, abort, lim))) break;
                         tc_fence_after();
                         if (MIXED && ((f >> x) & 1)) {
                             if ((x == 0 || !(f & 1)) && !(ok = pp_wait(&s.vb_full, bv & 1, abort, lim))) break;
                             tc_fence_after();
+                            const uint64_t dpb = make_sdesc(smem_u32(&s.pb[0][0]), 1024, 16, 2);
+                            const uint64_t dvb = make_sdesc(smem_u32(&s.vb[0][0]), 1024, 16384, 2);
+#pragma unroll
                             for (int ks = 0; ks < 8; ks++)
                                 mma_bf16(tbase + PP_O + PP_OW * x,
-                                         make_sdesc(smem_u32(s.pb[ks >> 2]) + 32 * (ks & 3), 1024, 16, 2),
-                                         make_sdesc(smem_u32(s.vb[0]) + 2048 * ks, 1024, 16384, 2),
-                                         idesc_bf16(128, D, 1), (u > 0 || ks > 0) ? 1u : 0u);
-                            // hand the bf16 P buffer to the next bf16 block once this P V completes
-                            if (++nx.x == 2) {
-                                nx.x = 0;
-                                nx.u++;
-                            }
-                            nx_st = pp_next_bf16_block<MIXED>(nx, p, nitems, nrounds, 1 << 30);
-                            if (nx_st == 1) tc_commit(&s.pb_grant[nx.x]);
+                                         dpb + (uint64_t)(((ks >> 2) * 16384 + 32 * (ks & 3)) >> 4),
+                                         dvb + (uint64_t)((2048 * ks) >> 4), idesc_bf16(128, D, 1),
+                                         (u > 0 || ks > 0) ? 1u : 0u);
                             if (x == 1 || !(f & 2)) {  // last bf16 P V of this key tile
                                 tc_commit(&s.vb_empty);
                                 bv++;
@@ -740,6 +769,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     tc_commit(&s.kv_empty[st]);  // this tile's P V are issued (the second release)
                 }
                 g0 += I.nu;
+                it++;
             }
             tc_commit(&s.drain);
             pp_drain(&s.drain, 0);
@@ -760,6 +790,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
         bool ok = true;
         int k = 0;   // key-tile steps of this tile so far (all items)
         int nb = 0;  // this tile's bf16 blocks so far
+        int bq_pos = 0, it = -1;  // read position in the bf16 tile queue; items so far
         int xp = 0;  // half-row exchanges so far
         // post this half's value of row r and return the other half's (bounded
         // wait: both halves count the same exchanges, two slots alternate)
@@ -767,6 +798,10 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             s.xch[xp & 1][x][h][r] = v;
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.xbar[x][quad]);
+            // the partner half is normally a few instructions away: poll briefly
+            // before a suspending wait
+            for (int n = 0; n < 32 && !mbar_test(&s.xbar[x][quad], xp & 1); n++) {
+            }
             if (!pp_wait(&s.xbar[x][quad], xp & 1, abort, lim)) return false;
             other = s.xch[xp & 1][x][h ^ 1][r];
             xp++;
@@ -776,67 +811,50 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             const int i = pp_item_index(j, nitems);
             if (i < 0) continue;
             const PpItem I = pp_item(p, i);
+            it++;
             const int nux = x == 0 ? I.nuA : I.nuB;
             const int tq = 2 * I.pair + x;
             const int row = tq * 128 + r;
             float crow = 0.0f;  // c_i = q_i . mean(K) for this row's bf16 scores
-            if (MIXED && nux > 0 && p.k_mean) {
-                const uint4* qr = reinterpret_cast<const uint4*>(p.q_bf16 + ((size_t)I.bh * p.N + min(row, p.N - 1)) * D);
-                const float* mu = p.k_mean + (size_t)I.bh * D;
-#pragma unroll 4
-                for (int c8 = 0; c8 < D / 8; c8++) {
-                    const uint4 w = __ldg(qr + c8);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        crow = __fmaf_rn(bf16_bits_to_f32(ww[e] & 0xFFFFu), __ldg(mu + 8 * c8 + 2 * e), crow);
-                        crow = __fmaf_rn(bf16_bits_to_f32(ww[e] >> 16), __ldg(mu + 8 * c8 + 2 * e + 1), crow);
-                    }
-                }
-            }
+            if (MIXED && nux > 0 && p.k_mean)
+                crow = pp_row_offset(p.q_bf16 + ((size_t)I.bh * p.N + min(row, p.N - 1)) * D,
+                                     p.k_mean + (size_t)I.bh * D, D);
             float m2 = -INFINITY;
             float lb = 0.0f;  // this half's share of the bf16 row sum (units of 2688 / g_V)
-            PpFlags fl{-64, 0, 0};
             for (int u = 0; u < nux; u++, k++) {
-                const bool bfx = MIXED && ((pp_flags<MIXED>(fl, p, I, u) >> x) & 1u);
                 if (!pp_wait(&s.s_full[x], k & 1, abort, lim)) {
                     ok = false;
                     break;
                 }
+                const bool bfx = MIXED && ((pp_bf16_flags<MIXED>(s, bq_pos, it, u) >> x) & 1u);
                 tc_fence_after();
                 float sv[64];
                 tmem_ld32(tbase + lane_off + PP_S + 64 * h, *reinterpret_cast<float(*)[32]>(&sv[0]));
                 tmem_ld32(tbase + lane_off + PP_S + 64 * h + 32, *reinterpret_cast<float(*)[32]>(&sv[32]));
                 tmem_wait_ld();
                 reg_fence(sv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.s_free[x]);
+                if (!(MIXED && bfx)) {  // a bf16 block re-reads S below and releases it then
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.s_free[x]);
+                }
 
                 const int kbase = u * 128 + 64 * h;
-                float hm;  // this half's max (raw S units for NVFP4, log2 units for bf16)
-                float bmax[4];
-                if (MIXED && bfx) {
-                    hm = -INFINITY;
+                const bool edge = (p.causal && u == tq) || (u * 128 + 128 > p.N);  // keys to mask
+                if (edge) {
 #pragma unroll
                     for (int i2 = 0; i2 < 64; i2++) {
                         const int key = kbase + i2;
-                        const bool valid = key < p.N && (!p.causal || key <= row);
-                        sv[i2] = valid ? __fsub_rn(sv[i2], crow) * cb : -INFINITY;
-                        hm = fmaxf(hm, sv[i2]);
+                        if (key >= p.N || (p.causal && key > row)) sv[i2] = -INFINITY;
                     }
-                } else {
-                    if ((p.causal && u == tq) || (u * 128 + 128 > p.N)) {
-#pragma unroll
-                        for (int i2 = 0; i2 < 64; i2++) {
-                            const int key = kbase + i2;
-                            if (key >= p.N || (p.causal && key > row)) sv[i2] = -INFINITY;
-                        }
-                    }
-#pragma unroll
-                    for (int blk = 0; blk < 4; blk++) bmax[blk] = pp_max16(&sv[16 * blk]);
-                    hm = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
                 }
+                float bmax[4];
+#pragma unroll
+                for (int blk = 0; blk < 4; blk++) bmax[blk] = pp_max16(&sv[16 * blk]);
+                // this half's max: raw S units for NVFP4; for a bf16 block the log2-unit
+                // score (S - c_i) sm_scale log2(e), a monotone map of S, so the max maps
+                float hm = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
+                if (MIXED && bfx && hm != -INFINITY) hm = __fsub_rn(hm, crow) * cb;
                 // the two halves agree on the row max
                 float om;
                 if (!exchange(hm, om)) {
@@ -849,30 +867,32 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 const float alpha = ex2f(m2 - msub);
                 m2 = m2_new;
 
-                uint32_t codes[8];
-                uint32_t scw = 0;
-                uint32_t pw[MIXED ? 32 : 1];
                 if (MIXED && bfx) {
-                    // P^ = bf16(2^(t - m)) as the method rounds it, then P' = bf16(P^ kappa)
-                    // in the NVFP4 accumulator's units (kappa = 2688 / g_V); the row sum
-                    // of P' is kept per half
-                    float ls = 0.0f;
-#pragma unroll
-                    for (int i2 = 0; i2 < 32; i2++) {
-                        const __nv_bfloat162 ph =
-                            __floats2bfloat162_rn(ex2f(sv[2 * i2] - msub), ex2f(sv[2 * i2 + 1] - msub));
-                        const __nv_bfloat162 pr =
-                            __floats2bfloat162_rn(__low2float(ph) * kappa, __high2float(ph) * kappa);
-                        ls += __low2float(pr);
-                        ls += __high2float(pr);
-                        pw[i2] = *reinterpret_cast<const uint32_t*>(&pr);
+                    // bf16 block: wait for the buffers first, then write P eight keys
+                    // at a time (no array of packed P held across the waits).  O is free
+                    // once this tile's previous P V finished; the shared bf16 P buffer
+                    // once the bf16 block before this one (either tile) finished its P V.
+                    if ((k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) ||
+                        !pp_wait(&s.pb_grant[x], nb & 1, abort, lim)) {
+                        ok = false;
+                        break;
                     }
+                    nb++;
+                    tc_fence_after();
+                    const float ls = pp_bf16_p_row(s.pb[h] + (r >> 3) * 1024 + (r & 7) * 128,
+                                                   tbase + lane_off + PP_S + 64 * h, r & 7, kbase, edge, p.N,
+                                                   p.causal != 0, row, crow, cb, msub, kappa);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.s_free[x]);  // S is read
                     lb = lb * alpha + ls;
+                    if (u == 0 && h == 1) tmem_st1(o_col + 128, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
                 } else {
                     // block scales first: E4M3 of (block max of P * 2688) / 6, and log2 of
                     // the scale value from a table
                     const float lm = kLog2_2688 - msub;
                     float bias[4];
+                    uint32_t scw = 0;
 #pragma unroll
                     for (int bp = 0; bp < 4; bp += 2) {
                         const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
@@ -886,6 +906,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                         }
                     }
                     // y = P * 2688 / scale, rounded to E2M1
+                    uint32_t codes[8];
 #pragma unroll
                     for (int c8 = 0; c8 < 8; c8++) {
                         const float* sp = &sv[8 * c8];
@@ -896,29 +917,13 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                                                ex2f(fmaf(sp[6], c2, bs)), ex2f(fmaf(sp[7], c2, bs)));
                     }
                     if (MIXED) lb *= alpha;
-                }
-                // P buffer and O are free once this tile's previous P V finished
-                // (for u = 0 that is the previous item's last one)
-                if (k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (MIXED && bfx) {
-                    // the bf16 P buffer is this block's once the bf16 block before it
-                    // (either tile) has finished its P V
-                    if (!pp_wait(&s.pb_grant[x], nb & 1, abort, lim)) {
+                    // P buffer and O are free once this tile's previous P V finished
+                    // (for u = 0 that is the previous item's last one)
+                    if (k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) {
                         ok = false;
                         break;
                     }
-                    nb++;
-                    uint8_t* prow = s.pb[h] + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int cc = 0; cc < 8; cc++)
-                        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
-                            make_uint4(pw[4 * cc], pw[4 * cc + 1], pw[4 * cc + 2], pw[4 * cc + 3]);
-                    if (u == 0 && h == 1) tmem_st1(o_col + 128, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
-                } else {
+                    tc_fence_after();
                     uint8_t* prow = s.p[x] + (r >> 3) * 512 + (r & 7) * 64;
 #pragma unroll
                     for (int c = 0; c < 2; c++) {

@@ -133,7 +133,10 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     float m2[kDecN];
 #pragma unroll
     for (int h = 0; h < kDecN; h++) m2[h] = -INFINITY;
-    if (tid < kDecN) s.mnew[tid] = -INFINITY;  // read after the first tile's barriers
+    if (tid < kDecN) {  // read after the first tile's barriers; padding columns stay at alpha 1
+        s.mnew[tid] = tid < p.G ? -INFINITY : 0.0f;
+        s.alpha[tid] = 1.0f;
+    }
     const int key0 = split * kSplit;
     const int nkeys = min(kSplit, p.L - key0);
     const int ntiles = nkeys / 128;
@@ -175,16 +178,17 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
 #pragma unroll
             for (int h = 0; h < kDecN; h++) sv[h] = __uint_as_float(r[h]);
         }
-        // column max over the 128 keys
+        // column max over the 128 keys (columns past the group's G heads are padding)
 #pragma unroll
         for (int h = 0; h < kDecN; h++) {
+            if (h >= p.G) break;
             float mx = sv[h];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             if (lane == 0) s.red[warp][h] = mx;
         }
         __syncthreads();
-        if (tid < kDecN) {
+        if (tid < p.G) {
             const float tmax = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
             const float mo = s.mnew[tid];  // the running max (-inf before the first tile)
             const float mn = fmaxf(mo, tmax * cexp);
@@ -201,6 +205,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         // P^T codes and scales: block of 16 keys = 16 lanes
 #pragma unroll
         for (int h = 0; h < kDecN; h++) {
+            if (h >= p.G) break;  // padding columns keep P = 0 (their O columns are not read)
             const float x = fmaf(sv[h], cexp, kLog2_2688 - m2[h]);
             float bm = x;
 #pragma unroll
@@ -253,7 +258,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (tid < kDecN) {  // l = alpha l + sum of this tile's dequantised P (warps in order)
+        if (tid < p.G) {  // l = alpha l + sum of this tile's dequantised P (warps in order)
             const float t = (s.lred[0][tid] + s.lred[1][tid]) + (s.lred[2][tid] + s.lred[3][tid]);
             s.lrun[tid] = (u > 0 ? s.lrun[tid] * s.alpha[tid] : 0.0f) + t;
         }

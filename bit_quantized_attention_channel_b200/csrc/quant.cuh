@@ -36,9 +36,13 @@ constexpr int kTile = 128;
 // Block quantisation (device)
 // ---------------------------------------------------------------------------
 
-// x / 6 rounded to nearest even.  For x >= 2^-120 the product by RN(1/6)
-// corrected by one FMA residual step equals the IEEE quotient (checked
-// exhaustively over every float in that range); smaller x divide directly.
+// x / 6 rounded to nearest even.  Method: P. Markstein's FMA correction of a
+// reciprocal-product quotient ("Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): q0 = RN(x y) with
+// y = RN(1/6), the remainder r = x - 6 q0 exact in one FMA, then
+// q = RN(q0 + r y).  For x >= 2^-120 this equals the IEEE quotient (checked
+// exhaustively over every float in that range against the hardware's
+// correctly rounded division); smaller x divide directly.
 SA_DEV float div6_rn(float x)
 {
     if (x < 7.52316384526264e-37f) return __fdiv_rn(x, 6.0f);  // 2^-120

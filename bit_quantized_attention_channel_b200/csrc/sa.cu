@@ -631,7 +631,29 @@ constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
+// per device: the scratch address and the context it was resolved in (a
+// device reset creates a new context, where the module and its array may sit
+// elsewhere, so the address is looked up again)
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+CUcontext g_noalloc_ctx[kNoAllocMaxDevices] = {};
+
+// The current driver context, through the runtime's driver entry point (no
+// link-time dependency on the driver library); null if unavailable.
+CUcontext current_context()
+{
+    using Fn = CUresult (*)(CUcontext*);
+    static const Fn fn = [] {
+        cudaDriverEntryPointQueryResult q;
+        void* ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<Fn>(ptr);
+        return (Fn) nullptr;
+    }();
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
 }  // namespace
 
 extern "C" sa_status sa_quant_nvfp4_noalloc(const void* x_dev, int B, int H, int N, int D, sa_role role, int smooth,
@@ -650,13 +672,15 @@ extern "C" sa_status sa_quant_nvfp4_noalloc(const void* x_dev, int B, int H, int
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_ptr[dev]) {
+        const CUcontext ctx = current_context();
+        if (!g_noalloc_ptr[dev] || !ctx || ctx != g_noalloc_ctx[dev]) {
             void* ptr = nullptr;
             if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
                 cudaGetLastError();
                 return SA_ERR_CUDA;
             }
             g_noalloc_ptr[dev] = ptr;
+            g_noalloc_ctx[dev] = ctx;
         }
         scratch = g_noalloc_ptr[dev];
     }

@@ -196,6 +196,17 @@ SA_DEV void tmem_st32(uint32_t taddr, const float (&v)[32])
         "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+// 8 consecutive columns of this thread's lane (completes before returning).
+SA_DEV void tmem_ld8_sync(uint32_t taddr, float (&v)[8])
+{
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
 SA_DEV float tmem_ld1(uint32_t taddr)
 {
     uint32_t r;

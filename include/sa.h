@@ -178,11 +178,14 @@ sa_status sa_quant_nvfp4_qkv(const void* q_dev, const void* k_dev, const void* v
  * held on every GPU that loads the library until the process exits.
  *  - Limit: sa_quant_workspace_size(B,H,N,D,role) must be <= 8 MiB, else
  *    SA_ERR_WORKSPACE is returned before anything is launched.  Q and V need
- *    256 bytes; K needs about 16*B*H*ceil(N/128)*D + 4*B*H*D bytes more
- *    (e.g. B*H*ceil(N/128) <= 3900 at D = 128).
- *  - The first call on a device looks up the scratch address for that
- *    device (cudaGetSymbolAddress, with the device current); make that first
- *    call before any stream capture.
+ *    256 bytes.  K needs 256 + a(8*B*H*T*D) + 2*a(4*B*H*T*D) + a(4*B*H*D)
+ *    bytes, T = ceil(N/128) and a() rounding up to a multiple of 256 (about
+ *    16*B*H*T*D bytes: at D = 128, B*H*T up to about 4080, the exact figure
+ *    depending on B*H; sa_quant_workspace_size gives it for any shape).
+ *  - The first call on a device (and the first after a reset of that device)
+ *    looks up the scratch address for the device's current context
+ *    (cudaGetSymbolAddress, with the device current); make that call before
+ *    any stream capture.
  *  - Calls share the scratch and it keeps the last call's contents; the call
  *    clears what must start at zero.  Calls that overlap on the GPU (for
  *    example on two streams at once) race: serialise them.

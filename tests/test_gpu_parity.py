@@ -94,6 +94,9 @@ def quality(got, ref):
 
 
 def sample_rows(N):
+    """Rows compared at full size: edge query tiles {0, 1, T/2, T-2, T-1} at
+    offsets {0, 1, 63, 64, 127}, plus 4 seeded random tiles at 8 offsets
+    (the rows are the same for every head)."""
     T = (N + 127) // 128
     rows = set()
     for t in sorted({0, 1, T // 2, T - 2, T - 1}):
@@ -101,6 +104,12 @@ def sample_rows(N):
             continue
         for o in (0, 1, 63, 64, 127):
             r = t * 128 + o
+            if r < N:
+                rows.add(r)
+    rng = np.random.default_rng(N)
+    for t in rng.choice(T, size=min(4, T), replace=False):
+        for o in (0, 17, 31, 32, 64, 95, 100, 127):
+            r = int(t) * 128 + o
             if r < N:
                 rows.add(r)
     return np.array(sorted(rows), np.int32)
@@ -310,7 +319,9 @@ def test_decode_full_size_sampled():
     q, k, v = wl.decode_inputs("decode")
     og = run_decode(q, k, v)
     ko, vo = orc.quantize(k, "k"), orc.quantize(v, "v")
-    pairs = np.array([0, 1, 5, 31, 32 * 7 + 3, 32 * 16 + 17, 32 * 31 + 30, 32 * 32 - 1], np.int32)
+    fixed = [0, 1, 5, 31, 32 * 7 + 3, 32 * 16 + 17, 32 * 31 + 30, 32 * 32 - 1]
+    extra = np.random.default_rng(4).choice(32 * 32, size=24, replace=False)
+    pairs = np.array(sorted(set(fixed) | {int(e) for e in extra}), np.int32)
     ref = orc.decode(q, ko, vo, pairs=pairs)
     check_close(og.reshape(-1, 128)[pairs], ref, "decode full")
 
