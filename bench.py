@@ -8,12 +8,14 @@ Metric: FP4 attention TOPS = 4*B*H*N^2*D / t (causal halved), t = step time.
 
 The headline workload is the long-context mixed-precision prefill (B1 H32
 N65536 D128 causal, top 5% of blocks in bf16), the largest configuration that
-fits one GPU; the LLM prefill (max-scaling and ScaleSearch), the video-shaped
-prefill and the NVFP4-KV decode are measured in the same run and nested in the
+fits one GPU; the LLM prefill (max-scaling, ScaleSearch on Q, K and V, and
+ScaleSearch on Q, K, V and P), the video-shaped
+prefill and the NVFP4-KV decode (plain, and with the cache's first and last
+128-key tile at full precision) are measured in the same run and nested in the
 line under "workloads".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME [--only]]
-                  [--mode max|search] [--impl ours|reference]
+                  [--mode max|search|psearch|sink] [--impl ours|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica (the path has no
 cross-GPU exchange), timing is the max over ranks, value is the job total.
@@ -157,7 +159,8 @@ class Path:
         if w.kind == "decode":
             return  # the KV cache is quantised once, before timing (it is a cache)
         # Q, K (smoothed) and V in two launches: statistics, then quantisation
-        st["qkv"] = sa.sa_quant_nvfp4_qkv(self.q, self.k, self.v, smooth=True, mode=self.mode, out=st.get("qkv"))
+        st["qkv"] = sa.sa_quant_nvfp4_qkv(self.q, self.k, self.v, smooth=True, mode=prepass_mode(self.mode),
+                                          out=st.get("qkv"))
         st["q"], st["k"], st["v"] = st["qkv"]
         if w.thrift_bp:
             st["mask"], _ = sa.sa_thrift_select(self.q, self.k, w.causal, w.thrift_bp)
@@ -165,18 +168,23 @@ class Path:
     def attention(self):
         w, st = self.w, self.st
         if w.kind == "decode":
-            st["o"] = sa.sa_attn_decode_kvfp4(self.q, st["kc"], st["vc"], out=st.get("o"))
+            st["o"] = sa.sa_attn_decode_kvfp4(self.q, st["kc"], st["vc"], out=st.get("o"),
+                                              sink_tiles=sink_tiles(self.mode), k_sink=st.get("ks"),
+                                              v_sink=st.get("vs"))
         elif w.thrift_bp:
             st["o"] = sa.sa_attn_fwd(st["q"], st["k"], st["v"], w.causal, mask=st["mask"], q_bf16=self.q,
                                      k_bf16=self.k, v_bf16=self.v, out=st.get("o"))
         else:
-            st["o"] = sa.sa_attn_fwd(st["q"], st["k"], st["v"], w.causal, out=st.get("o"))
+            st["o"] = sa.sa_attn_fwd(st["q"], st["k"], st["v"], w.causal, out=st.get("o"), p_mode=p_mode(self.mode))
         return st["o"]
 
     def setup(self):
         if self.w.kind == "decode":
             self.st["kc"] = sa.sa_quant_nvfp4(self.k, "k")
             self.st["vc"] = sa.sa_quant_nvfp4(self.v, "v")
+            if any(sink_tiles(self.mode)):  # the cache's full-precision first and last tiles
+                self.st["ks"] = sa.sink_tiles_of(self.k, *sink_tiles(self.mode))
+                self.st["vs"] = sa.sink_tiles_of(self.v, *sink_tiles(self.mode))
 
     def capture(self):
         """Warm up eagerly, then capture both phases as CUDA graphs."""
@@ -202,6 +210,23 @@ class Path:
         return self.st["o"]
 
 
+def prepass_mode(mode):
+    """Block rule of the pre-pass: "search" and "psearch" use ScaleSearch."""
+    return "search" if mode in ("search", "psearch") else "max"
+
+
+def p_mode(mode):
+    """Block rule of the requantised P: ScaleSearch only in mode "psearch"
+    (Q, K, V and P all ScaleSearch)."""
+    return "search" if mode == "psearch" else "max"
+
+
+def sink_tiles(mode):
+    """Decode mode "sink": the first and the last 128-key tile of the cache
+    at full precision (the attention-sink-aware mixed-precision cache)."""
+    return (1, 1) if mode == "sink" else (0, 0)
+
+
 def kernels_per_step(w):
     if w.kind == "decode":
         return 3  # q amax, split kernel, combine
@@ -217,10 +242,12 @@ def flops_of(w):
     return w.flops()
 
 
-def hbm_bytes_decode(w):
-    """Algorithmic bytes of one decode: K and V codes + scales, q, out."""
-    kv = 2 * (w.B * w.Hkv * w.N * w.D // 2 + w.B * w.Hkv * w.N * w.D // 16)
-    return kv + w.B * w.H * w.D * (2 + 4)
+def hbm_bytes_decode(w, mode="max"):
+    """Algorithmic bytes of one decode: K and V codes + scales, q, out; with
+    full-precision tiles, their bf16 K and V in place of their NVFP4 bytes."""
+    nsink = 128 * sum(sink_tiles(mode))
+    kv = 2 * w.B * w.Hkv * ((w.N - nsink) * w.D * 0.5625 + nsink * w.D * 2)
+    return int(kv) + w.B * w.H * w.D * (2 + 4)
 
 
 def prepass_bytes(w):
@@ -247,7 +274,7 @@ def cpu_sample_step(w, mode, q, k, v, tiles):
 
     import oracle as orc
 
-    ss = mode == "search"
+    ss = prepass_mode(mode) == "search"
     N, D = w.N, w.D
     t0 = time.perf_counter()
     qo, ko, vo = orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss), orc.quantize(v, "v", search=ss)
@@ -260,7 +287,7 @@ def cpu_sample_step(w, mode, q, k, v, tiles):
     if mask is not None:
         orc.attention(qo, ko, vo, w.causal, rows=rows, mask=mask, q_bf16=q, k_bf16=k, v_bf16=v)
     else:
-        orc.attention(qo, ko, vo, w.causal, rows=rows)
+        orc.attention(qo, ko, vo, w.causal, rows=rows, p_search=p_mode(mode) == "search")
     t_attn = time.perf_counter() - t1
     keys = float((rows + 1).sum()) if w.causal else float(len(rows)) * N
     flops = 4.0 * keys * D
@@ -354,18 +381,22 @@ def traffic_of(w, kname, args):
 
 def config_of(w, mode):
     c = {"workload": w.description, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "causal": w.causal,
-         "scale_mode": mode, "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
+         "scale_mode": prepass_mode(mode), "p_scale_mode": p_mode(mode), "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
          "launch": "CUDA graphs (pre-pass graph + attention graph per step)"}
     if w.kind == "decode":
         c["Hkv"] = w.Hkv
+        c["scale_mode"] = "max"
+        c["sink_tiles"] = list(sink_tiles(mode))
     if w.thrift_bp:
         c["bf16_block_budget_bp"] = w.thrift_bp
     return c
 
 
-def kernel_name(w):
+def kernel_name(w, mode="max"):
     if w.kind == "decode":
-        return "decode_kernel<128> + combine"
+        return "decode_kernel<128, sink> + combine" if any(sink_tiles(mode)) else "decode_kernel<128> + combine"
+    if p_mode(mode) == "search":
+        return "attn_fwd_pp_kernel<128, P ScaleSearch>"
     return "attn_fwd_pp_kernel<128, mixed>" if w.thrift_bp else "attn_fwd_pp_kernel<128>"
 
 
@@ -416,13 +447,13 @@ def measure(w, mode, args, dev, pg, world, flush, want_e2e=True):
     hbm, bf16, src = peaks()
     fp4_peak = bf16 * 4.0  # dense FP4 = 4x dense bf16 (nominal ratio 9 / 2.25)
     flops = flops_of(w)
-    kname = kernel_name(w)
+    kname = kernel_name(w, mode)
     if w.kind == "decode":
-        gbs = hbm_bytes_decode(w) / (ms_attn * 1e-3) / 1e9
+        gbs = hbm_bytes_decode(w, mode) / (ms_attn * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                 "peak_source": f"{src} copy bandwidth", "traffic": traffic_of(w, kname, args),
                 "traffic_unit": "DRAM bytes per launch (ncu, batch slice scaled)", "ms_per_launch": ms_attn,
-                "algorithmic_bytes": hbm_bytes_decode(w)}
+                "algorithmic_bytes": hbm_bytes_decode(w, mode)}
         value = whole_job_tops(world, flops, ms)
     else:
         achieved = flops / (ms_attn * 1e-3) / 1e12
@@ -461,7 +492,7 @@ def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
     e2e_paths, houts = [], []
     for _ in range(2):
         pth = Path(w, mode, torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-        pth.st.update({kk: path.st[kk] for kk in ("kc", "vc") if kk in path.st})
+        pth.st.update({kk: path.st[kk] for kk in ("kc", "vc", "ks", "vs") if kk in path.st})
         e2e_paths.append(pth)
         houts.append(torch.empty(path.st["o"].shape, dtype=torch.float32).pin_memory())
 
@@ -519,7 +550,8 @@ def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
 # largest configuration that fits one GPU (the long-context mixed prefill);
 # the others are measured in the same run and nested in the line.
 HEADLINE = ("longctx", "max")
-OTHERS = [("llm", "max"), ("llm", "search"), ("video", "search"), ("decode", "max")]
+OTHERS = [("llm", "max"), ("llm", "search"), ("llm", "psearch"), ("video", "search"), ("decode", "max"),
+          ("decode", "sink")]
 
 
 def main():
@@ -528,7 +560,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=HEADLINE[0])
-    ap.add_argument("--mode", default=None, choices=["max", "search"])
+    ap.add_argument("--mode", default=None, choices=["max", "search", "psearch", "sink"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only", action="store_true", help="measure the named workload alone (no nested workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

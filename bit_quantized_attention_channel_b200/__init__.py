@@ -12,7 +12,8 @@ Entry points keep the C names:
   sa_thrift_select      high-precision block selector
   sa_thrift_select_ex   the selector with per-row budgets / smoothed-K pooling
   sa_attn_fwd           NVFP4 attention forward (optionally with bf16 blocks)
-  sa_attn_decode_kvfp4  decode over an NVFP4 KV cache
+  sa_attn_decode_kvfp4  decode over an NVFP4 KV cache (optionally with
+                        full-precision first/last tiles)
 """
 from __future__ import annotations
 
@@ -71,6 +72,10 @@ def lib():
         L.sa_decode_workspace_size.argtypes, L.sa_decode_workspace_size.restype = [I, I, I, I, I], Z
         L.sa_attn_decode_kvfp4.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, Z, P]
         L.sa_attn_decode_kvfp4.restype = I
+        L.sa_attn_decode_kvfp4_sink.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]
+        L.sa_attn_decode_kvfp4_sink.restype = I
+        L.sa_attn_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, P, P, P, P, P, P, P]
+        L.sa_attn_fwd_ex.restype = I
         _lib = L
     return _lib
 
@@ -290,8 +295,11 @@ def sa_thrift_select_ex(q, k, causal: bool, frac_bp: int = 500, per_row: bool = 
 
 
 def sa_attn_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, causal: bool, sm_scale: float = 0.0, mask=None,
-                q_bf16=None, k_bf16=None, v_bf16=None, want_lse: bool = False, out=None, stream=None):
-    """FP32 attention output [B,H,N,D] (and lse [B,H,N] if asked)."""
+                q_bf16=None, k_bf16=None, v_bf16=None, want_lse: bool = False, out=None, stream=None,
+                p_mode: str = "max"):
+    """FP32 attention output [B,H,N,D] (and lse [B,H,N] if asked).
+    p_mode: block rule of the requantised P, "max" (max-scaling) or
+    "search" (ScaleSearch; sa_attn_fwd_ex)."""
     import torch
 
     _nvfp4("q", q, v_layout=False)
@@ -314,16 +322,29 @@ def sa_attn_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, causal: bool, sm
         out = torch.empty(B, H, N, D, dtype=torch.float32, device=dev)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_lse else None
     km = k.k_mean if mask is not None else None
-    _check("sa_attn_fwd",
-           lib().sa_attn_fwd(_ptr(q.codes), _ptr(q.scales), _ptr(q.g), _ptr(k.codes), _ptr(k.scales), _ptr(k.g),
-                             _ptr(v.codes), _ptr(v.scales), _ptr(v.g), B, H, N, D, int(causal), float(sm_scale),
-                             _ptr(mask), _ptr(q_bf16), _ptr(k_bf16), _ptr(v_bf16), _ptr(km), _ptr(out), _ptr(lse),
-                             _stream(stream)))
+    pm = _mode(p_mode)
+    if pm == 0:
+        _check("sa_attn_fwd",
+               lib().sa_attn_fwd(_ptr(q.codes), _ptr(q.scales), _ptr(q.g), _ptr(k.codes), _ptr(k.scales),
+                                 _ptr(k.g), _ptr(v.codes), _ptr(v.scales), _ptr(v.g), B, H, N, D, int(causal),
+                                 float(sm_scale), _ptr(mask), _ptr(q_bf16), _ptr(k_bf16), _ptr(v_bf16), _ptr(km),
+                                 _ptr(out), _ptr(lse), _stream(stream)))
+    else:
+        _check("sa_attn_fwd_ex",
+               lib().sa_attn_fwd_ex(_ptr(q.codes), _ptr(q.scales), _ptr(q.g), _ptr(k.codes), _ptr(k.scales),
+                                    _ptr(k.g), _ptr(v.codes), _ptr(v.scales), _ptr(v.g), B, H, N, D, int(causal),
+                                    float(sm_scale), pm, _ptr(mask), _ptr(q_bf16), _ptr(k_bf16), _ptr(v_bf16),
+                                    _ptr(km), _ptr(out), _ptr(lse), _stream(stream)))
     return (out, lse) if want_lse else out
 
 
-def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.0, out=None, stream=None):
-    """q bf16 [B,Hq,D]; caches quantised as [B,Hkv,L,D]; returns FP32 [B,Hq,D]."""
+def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.0, out=None, stream=None,
+                         sink_tiles=(0, 0), k_sink=None, v_sink=None):
+    """q bf16 [B,Hq,D]; caches quantised as [B,Hkv,L,D]; returns FP32 [B,Hq,D].
+    sink_tiles = (first, last) keeps that many 128-key tiles at each end of
+    the cache at full precision (sa_attn_decode_kvfp4_sink); k_sink, v_sink
+    are then bf16 [B,Hkv,128 (first + last),D] holding those tiles, and the
+    channel means of k (k.k_mean) offset their keys."""
     import torch
 
     _bf16("q", q, 3)
@@ -337,16 +358,43 @@ def sa_attn_decode_kvfp4(q, k: NVFP4Tensor, v: NVFP4Tensor, sm_scale: float = 0.
         _tensor("out", out, torch.float32, 3, (B, Hq, D))
     _on_device("k", k)
     _on_device("v", v)
+    first, last = (int(t) for t in sink_tiles)
+    if first < 0 or last < 0:
+        raise ValueError(f"sink_tiles: {sink_tiles}")
+    if first or last:
+        ns = 128 * (first + last)
+        _bf16("k_sink", k_sink, 4, (B, Hkv, ns, D))
+        _bf16("v_sink", v_sink, 4, (B, Hkv, ns, D))
     L = lib()
     if out is None:
         out = torch.empty(B, Hq, D, dtype=torch.float32, device=q.device)
     ws_bytes = L.sa_decode_workspace_size(B, Hq, Hkv, Lk, D)
     ws = _empty(ws_bytes, q.device)
-    _check("sa_attn_decode_kvfp4",
-           L.sa_attn_decode_kvfp4(_ptr(q), _ptr(k.codes), _ptr(k.scales), _ptr(k.g), _ptr(v.codes), _ptr(v.scales),
-                                  _ptr(v.g), B, Hq, Hkv, Lk, D, float(sm_scale), _ptr(out), _ptr(ws), ws_bytes,
-                                  _stream(stream)))
+    if first or last:
+        _check("sa_attn_decode_kvfp4_sink",
+               L.sa_attn_decode_kvfp4_sink(_ptr(q), _ptr(k.codes), _ptr(k.scales), _ptr(k.g), _ptr(v.codes),
+                                           _ptr(v.scales), _ptr(v.g), B, Hq, Hkv, Lk, D, float(sm_scale), first, last,
+                                           _ptr(k_sink), _ptr(v_sink), _ptr(k.k_mean), _ptr(out), _ptr(ws), ws_bytes,
+                                           _stream(stream)))
+    else:
+        _check("sa_attn_decode_kvfp4",
+               L.sa_attn_decode_kvfp4(_ptr(q), _ptr(k.codes), _ptr(k.scales), _ptr(k.g), _ptr(v.codes),
+                                      _ptr(v.scales), _ptr(v.g), B, Hq, Hkv, Lk, D, float(sm_scale), _ptr(out),
+                                      _ptr(ws), ws_bytes, _stream(stream)))
     return out
+
+
+def sink_tiles_of(x, first: int, last: int):
+    """The compact full-precision copy that sa_attn_decode_kvfp4 takes for
+    sink_tiles = (first, last): the first `first` and the last `last`
+    128-key tiles of a [B,Hkv,L,D] cache, concatenated along the keys."""
+    import torch
+
+    L = x.shape[2]
+    parts = [x[:, :, : 128 * first]] if first else []
+    if last:
+        parts.append(x[:, :, L - 128 * last:])
+    return torch.cat(parts, dim=2).contiguous()
 
 
 # --------------------------------------------------------------------- layouts

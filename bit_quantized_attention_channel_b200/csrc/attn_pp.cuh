@@ -46,6 +46,7 @@
 #pragma once
 
 #include "attn.cuh"
+#include "quant.cuh"
 
 namespace sa {
 
@@ -78,6 +79,7 @@ struct PpSmem {
     int4 bfq[16];
     int bfq_n;                // entries pushed
     float lg2sc[128];         // log2 of each nonzero E4M3 scale value
+    float rcp[128];           // 1 / each E4M3 scale value (ScaleSearch on P)
     float xch[2][2][2][128];  // half-row exchange: [use parity][tile][half][row]
     uint64_t q_full[QB];      // Q tiles and scale atoms landed
     uint64_t q_empty[QB];     // every Q K^T of the item completed
@@ -356,7 +358,7 @@ __device__ __noinline__ float pp_row_offset(const uint16_t* qrow, const float* m
     return c;
 }
 
-template <int D, bool MIXED>
+template <int D, bool MIXED, bool PSEARCH>
 __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                                     const __grid_constant__ CUtensorMap tm_k,
                                                                     const __grid_constant__ CUtensorMap tm_v,
@@ -423,6 +425,7 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
             tma_prefetch_desc(&tm_vb);
         }
     }
+    if (PSEARCH) fill_rcp_table(s.rcp);
     if (tid < 128) {
         // (e - 7) + log2(1 + m/8) for normal bytes, -7 + log2(m/4) for subnormal ones
         const uint32_t e = (uint32_t)tid >> 3, m = (uint32_t)tid & 7u;
@@ -888,33 +891,50 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     lb = lb * alpha + ls;
                     if (u == 0 && h == 1) tmem_st1(o_col + 128, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
                 } else {
-                    // block scales first: E4M3 of (block max of P * 2688) / 6, and log2 of
-                    // the scale value from a table
                     const float lm = kLog2_2688 - msub;
-                    float bias[4];
                     uint32_t scw = 0;
+                    uint32_t codes[8];
+                    if constexpr (PSEARCH) {
+                        // ScaleSearch on P ("Search Your Block Floating Point Scales!",
+                        // "ScaleSearch" applied to the requantised P): per 16 keys the block
+                        // rule of the pre-pass on p~ = P * 2688, scale codes c0 + f for f in
+                        // [-2, 6), the least squared error kept
 #pragma unroll
-                    for (int bp = 0; bp < 4; bp += 2) {
-                        const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
-                                                             ex2f(fmaf(bmax[bp + 1], c2, lm)) * (1.0f / 6.0f));
+                        for (int blk = 0; blk < 4; blk++) {
+                            float xt[16];
 #pragma unroll
-                        for (int hh = 0; hh < 2; hh++) {
-                            const int blk = bp + hh;
-                            const uint32_t sc = (sc2 >> (8 * hh)) & 0xFFu;
-                            bias[blk] = sc ? lm - s.lg2sc[sc] : -INFINITY;
+                            for (int i2 = 0; i2 < 16; i2++) xt[i2] = ex2f(fmaf(sv[16 * blk + i2], c2, lm));
+                            uint32_t sc;
+                            int off;
+                            quant16<true>(xt, -2, 6, codes[2 * blk], codes[2 * blk + 1], sc, off, s.rcp);
                             scw |= sc << (8 * blk);
                         }
-                    }
-                    // y = P * 2688 / scale, rounded to E2M1
-                    uint32_t codes[8];
+                    } else {
+                        // block scales first: E4M3 of (block max of P * 2688) / 6, and log2 of
+                        // the scale value from a table
+                        float bias[4];
 #pragma unroll
-                    for (int c8 = 0; c8 < 8; c8++) {
-                        const float* sp = &sv[8 * c8];
-                        const float bs = bias[c8 >> 1];
-                        codes[c8] = pack8_e2m1(ex2f(fmaf(sp[0], c2, bs)), ex2f(fmaf(sp[1], c2, bs)),
-                                               ex2f(fmaf(sp[2], c2, bs)), ex2f(fmaf(sp[3], c2, bs)),
-                                               ex2f(fmaf(sp[4], c2, bs)), ex2f(fmaf(sp[5], c2, bs)),
-                                               ex2f(fmaf(sp[6], c2, bs)), ex2f(fmaf(sp[7], c2, bs)));
+                        for (int bp = 0; bp < 4; bp += 2) {
+                            const uint32_t sc2 = f32x2_to_e4m3x2(ex2f(fmaf(bmax[bp], c2, lm)) * (1.0f / 6.0f),
+                                                                 ex2f(fmaf(bmax[bp + 1], c2, lm)) * (1.0f / 6.0f));
+#pragma unroll
+                            for (int hh = 0; hh < 2; hh++) {
+                                const int blk = bp + hh;
+                                const uint32_t sc = (sc2 >> (8 * hh)) & 0xFFu;
+                                bias[blk] = sc ? lm - s.lg2sc[sc] : -INFINITY;
+                                scw |= sc << (8 * blk);
+                            }
+                        }
+                        // y = P * 2688 / scale, rounded to E2M1
+#pragma unroll
+                        for (int c8 = 0; c8 < 8; c8++) {
+                            const float* sp = &sv[8 * c8];
+                            const float bs = bias[c8 >> 1];
+                            codes[c8] = pack8_e2m1(ex2f(fmaf(sp[0], c2, bs)), ex2f(fmaf(sp[1], c2, bs)),
+                                                   ex2f(fmaf(sp[2], c2, bs)), ex2f(fmaf(sp[3], c2, bs)),
+                                                   ex2f(fmaf(sp[4], c2, bs)), ex2f(fmaf(sp[5], c2, bs)),
+                                                   ex2f(fmaf(sp[6], c2, bs)), ex2f(fmaf(sp[7], c2, bs)));
+                        }
                     }
                     if (MIXED) lb *= alpha;
                     // P buffer and O are free once this tile's previous P V finished

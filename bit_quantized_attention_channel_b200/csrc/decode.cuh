@@ -19,6 +19,18 @@
 // pass (same block rule as the pre-pass: 16 channels, max-scaling).
 // Each split writes (m, l, O) unnormalised; decode_combine_kernel merges the
 // splits exactly: O = sum_s 2^(m_s-M) O_s / sum_s 2^(m_s-M) l_s.
+//
+// Attention-sink-aware mixed-precision cache (same page, "ScaleSearchAttention":
+// the first and last blocks of the cache stay at full precision): with SINK,
+// the first sink_first and the last sink_last 128-key tiles of the cache come
+// from a compact bf16 copy of just those tiles and take the mixed-block
+// arithmetic inside the same online softmax: scores of raw bf16 q against raw
+// bf16 k minus its channel mean, P~ rounded to bf16, raw bf16 V.  These tiles
+// are a few per cache and their MMA shape (128 keys x G heads) is mostly
+// padding, so they run on the CUDA cores with FP32 accumulation, reading K and
+// V straight from global memory; the kernel keeps the plain decode's shared
+// memory (and occupancy).  Their P·V adds into the TMEM accumulator in its
+// NVFP4 units: O += (2688 P_b) (V / g_V), l += 2688 P_b.
 #pragma once
 
 #include "attn.cuh"
@@ -78,9 +90,188 @@ struct DecParams {
     float* part;  // [B*Hq, nsplit, D + 2]: O (D), l, m
     int L, Hq, Hkv, G, nsplit, RTk, CKv;
     float sm_scale;
+    // full-precision tiles (SINK): bf16 [B, Hkv, NS, D], NS = 128 (sink_first + sink_last),
+    // the first tiles then the last ones; k_mean [B, Hkv, D] (nullptr: K not smoothed)
+    const uint16_t* k_sink;
+    const uint16_t* v_sink;
+    const float* k_mean;
+    int sink_first, sink_last, NS;
 };
 
+// One full-precision cache tile: thread tid holds key tid for the scores and
+// channel tid for P·V.  sv receives q.(k - mu) per head (h < G; padding
+// heads 0).  pbuf: 128 G floats of shared memory for P_b.
 template <int D>
+SA_DEV void dec_sink_scores(const DecParams& p, int b, int hk, int srow, float (&sv)[kDecN])
+{
+    const int tid = threadIdx.x;
+    const size_t kv = (size_t)b * p.Hkv + hk;
+    const uint4* krow = reinterpret_cast<const uint4*>(p.k_sink + (kv * p.NS + srow + tid) * D);
+    const float* mu = p.k_mean ? p.k_mean + kv * D : nullptr;
+    const uint16_t* qg = p.q + ((size_t)b * p.Hq + (size_t)hk * p.G) * D;
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) sv[h] = 0.0f;
+#pragma unroll 2
+    for (int c = 0; c < D / 8; c++) {
+        const uint4 kr = __ldg(krow + c);
+        const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
+        float kf[8];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            kf[2 * i] = __uint_as_float(kw[i] << 16);
+            kf[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
+        }
+        if (mu) {
+            const float4 m0 = __ldg(reinterpret_cast<const float4*>(mu + 8 * c));
+            const float4 m1 = __ldg(reinterpret_cast<const float4*>(mu + 8 * c + 4));
+            kf[0] -= m0.x, kf[1] -= m0.y, kf[2] -= m0.z, kf[3] -= m0.w;
+            kf[4] -= m1.x, kf[5] -= m1.y, kf[6] -= m1.z, kf[7] -= m1.w;
+        }
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) {
+            if (h >= p.G) break;
+            const uint4 qr = __ldg(reinterpret_cast<const uint4*>(qg + (size_t)h * D) + c);  // warp-uniform
+            const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w};
+            float a = sv[h];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                a = fmaf(__uint_as_float(qw[i] << 16), kf[2 * i], a);
+                a = fmaf(__uint_as_float(qw[i] & 0xFFFF0000u), kf[2 * i + 1], a);
+            }
+            sv[h] = a;
+        }
+    }
+}
+
+// O^T row d = tid (d < D) of a full-precision tile: sum over the 128 keys of
+// P_b[h][key] V[key][d] in FP32, returned per head.
+template <int D>
+SA_DEV void dec_sink_pv(const DecParams& p, int b, int hk, int srow, const float* pbuf, float (&acc)[kDecN])
+{
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) acc[h] = 0.0f;
+    if (tid >= D) return;
+    const size_t kv = (size_t)b * p.Hkv + hk;
+    const uint16_t* vcol = p.v_sink + (kv * p.NS + srow) * D + tid;
+#pragma unroll 1
+    for (int k0 = 0; k0 < 128; k0 += 8) {
+        float vv[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) vv[i] = __uint_as_float((uint32_t)__ldg(vcol + (size_t)(k0 + i) * D) << 16);
+#pragma unroll
+        for (int h = 0; h < kDecN; h++) {
+            if (h >= p.G) break;
+            float a = acc[h];
+#pragma unroll
+            for (int i = 0; i < 8; i += 4) {
+                const float4 pw = *reinterpret_cast<const float4*>(pbuf + h * 128 + k0 + i);  // broadcast
+                a = fmaf(pw.x, vv[i], a);
+                a = fmaf(pw.y, vv[i + 1], a);
+                a = fmaf(pw.z, vv[i + 2], a);
+                a = fmaf(pw.w, vv[i + 3], a);
+            }
+            acc[h] = a;
+        }
+    }
+}
+
+// Running max per column (query head) after one tile: max over the 128 keys
+// of sv * c (columns past the group's G heads are padding and keep m = 0,
+// alpha = 1).  Returns the new max m2 and the rescale factor alpha per column.
+template <int D>
+SA_DEV void dec_running_max(DecSmem<D>& s, const DecParams& p, const float (&sv)[kDecN], float c,
+                            float (&m2)[kDecN], float (&alpha)[kDecN])
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) {
+        if (h >= p.G) break;
+        float mx = sv[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) s.red[warp][h] = mx;
+    }
+    __syncthreads();
+    if (tid < p.G) {
+        const float tmax = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
+        const float mo = s.mnew[tid];  // the running max (-inf before the first tile)
+        const float mn = fmaxf(mo, tmax * c);
+        s.mnew[tid] = mn;
+        s.alpha[tid] = ex2f(mo - mn);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) {
+        m2[h] = s.mnew[h];
+        alpha[h] = s.alpha[h];
+    }
+}
+
+// l = alpha l + the tile's per-warp sums of P (warps in a fixed order).
+template <int D>
+SA_DEV void dec_l_update(DecSmem<D>& s, const DecParams& p, int u)
+{
+    const int tid = threadIdx.x;
+    if (tid < p.G) {
+        const float t = (s.lred[0][tid] + s.lred[1][tid]) + (s.lred[2][tid] + s.lred[3][tid]);
+        s.lrun[tid] = (u > 0 ? s.lrun[tid] * s.alpha[tid] : 0.0f) + t;
+    }
+}
+
+// The rest of a full-precision tile once its scores sv are known: running
+// max, P_b = bf16(2^(sv c - m)) into shared memory (the K tile's buffer,
+// unused by this tile), P·V on the CUDA cores, O^T = alpha O^T + kappa acc in
+// TMEM (kappa = 2688 / g_V, the accumulator's NVFP4 units), l += 2688 P_b.
+template <int D>
+SA_DEV bool dec_sink_tile(DecSmem<D>& s, const DecParams& p, int b, int hk, int srow, int u,
+                          const float (&sv)[kDecN], float c, uint32_t tbase, uint32_t lane_off)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float m2[kDecN], alpha[kDecN];
+    dec_running_max(s, p, sv, c, m2, alpha);
+    float* pbuf = reinterpret_cast<float*>(s.k);  // [G][128] (4 KB <= the K tile's bytes)
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) {
+        if (h >= p.G) break;
+        const float pb = __bfloat162float(__float2bfloat16_rn(ex2f(fmaf(sv[h], c, -m2[h]))));
+        pbuf[h * 128 + tid] = pb;
+        float pv = pb * 2688.0f;  // exact: 8 significant bits times 21 * 2^7
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pv += __shfl_xor_sync(0xffffffffu, pv, o);
+        if (lane == 0) s.lred[warp][h] = pv;
+    }
+    __syncthreads();
+    float acc[kDecN];
+    dec_sink_pv<D>(p, b, hk, srow, pbuf, acc);
+    const float kappa = 2688.0f / p.v_g[0];
+    uint32_t r[kDecN];
+    if (u > 0)
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+            : "r"(tbase + lane_off + DM_O)
+            : "memory");
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) {
+        const float o = u > 0 ? __uint_as_float(r[h]) * alpha[h] : 0.0f;
+        r[h] = __float_as_uint(fmaf(acc[h], kappa, o));
+    }
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(tbase + lane_off + DM_O),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+    fence_proxy_async();  // the K tile's buffer goes back to the tensor copies
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    dec_l_update(s, p, u);
+    return true;
+}
+
+template <int D, bool SINK>
 SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMap* tm_v, const DecParams& p,
                         int b, int hk, int split, uint32_t tbase)
 {
@@ -130,9 +321,6 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
     }
 
-    float m2[kDecN];
-#pragma unroll
-    for (int h = 0; h < kDecN; h++) m2[h] = -INFINITY;
     if (tid < kDecN) {  // read after the first tile's barriers; padding columns stay at alpha 1
         s.mnew[tid] = tid < p.G ? -INFINITY : 0.0f;
         s.alpha[tid] = 1.0f;
@@ -140,8 +328,26 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     const int key0 = split * kSplit;
     const int nkeys = min(kSplit, p.L - key0);
     const int ntiles = nkeys / 128;
+    const float c_sink = p.sm_scale * kLog2e;  // full-precision tiles: t = q.(k - mu) sm_scale log2(e)
     for (int u = 0; u < ntiles; u++) {
         const int ktile = key0 / 128 + u;
+        bool sink = false;
+        int srow = 0;
+        if constexpr (SINK) {
+            if (ktile < p.sink_first) {
+                sink = true;
+                srow = ktile * 128;
+            } else if (ktile >= p.RTk - p.sink_last) {
+                sink = true;
+                srow = (p.sink_first + ktile - (p.RTk - p.sink_last)) * 128;
+            }
+        }
+        if (sink) {
+            float sv[kDecN];
+            dec_sink_scores<D>(p, b, hk, srow, sv);
+            if (!dec_sink_tile<D>(s, p, b, hk, srow, u, sv, c_sink, tbase, lane_off)) return false;
+            continue;
+        }
         if (tid == 0) {
             mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + 2 * 512);
             tma_load_3d(s.k, tm_k, &s.tma_bar, 0, ktile * 128, bhk);
@@ -178,30 +384,9 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
 #pragma unroll
             for (int h = 0; h < kDecN; h++) sv[h] = __uint_as_float(r[h]);
         }
-        // column max over the 128 keys (columns past the group's G heads are padding)
-#pragma unroll
-        for (int h = 0; h < kDecN; h++) {
-            if (h >= p.G) break;
-            float mx = sv[h];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) s.red[warp][h] = mx;
-        }
-        __syncthreads();
-        if (tid < p.G) {
-            const float tmax = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
-            const float mo = s.mnew[tid];  // the running max (-inf before the first tile)
-            const float mn = fmaxf(mo, tmax * cexp);
-            s.mnew[tid] = mn;
-            s.alpha[tid] = ex2f(mo - mn);
-        }
-        __syncthreads();
         float alpha[kDecN];
-#pragma unroll
-        for (int h = 0; h < kDecN; h++) {
-            m2[h] = s.mnew[h];
-            alpha[h] = s.alpha[h];
-        }
+        float m2[kDecN];
+        dec_running_max(s, p, sv, cexp, m2, alpha);
         // P^T codes and scales: block of 16 keys = 16 lanes
 #pragma unroll
         for (int h = 0; h < kDecN; h++) {
@@ -258,10 +443,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (tid < p.G) {  // l = alpha l + sum of this tile's dequantised P (warps in order)
-            const float t = (s.lred[0][tid] + s.lred[1][tid]) + (s.lred[2][tid] + s.lred[3][tid]);
-            s.lrun[tid] = (u > 0 ? s.lrun[tid] * s.alpha[tid] : 0.0f) + t;
-        }
+        dec_l_update(s, p, u);
         if (tid == 0) {
             tc_fence_after();
             for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
@@ -287,20 +469,20 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         : "r"(tbase + lane_off + DM_O)
         : "memory");
 #pragma unroll
-    for (int h = 0; h < kDecN; h++) {  // constant indices keep o and m2 in registers
+    for (int h = 0; h < kDecN; h++) {  // constant indices keep o in registers
         if (h >= p.G) break;
         float* dst = p.part + (((size_t)b * p.Hq + hk * p.G + h) * p.nsplit + split) * (D + 2);
         if (tid < D) dst[tid] = __uint_as_float(o[h]);
         if (tid == 0) {
             dst[D] = s.lrun[h];
-            dst[D + 1] = m2[h];
+            dst[D + 1] = s.mnew[h];
         }
     }
     return true;
 }
 
-template <int D>
-__global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+template <int D, bool SINK>
+__global__ void __launch_bounds__(128, 8) decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                      const __grid_constant__ CUtensorMap tm_v, const DecParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -332,7 +514,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = s.tmem_slot;
-    if (!decode_body<D>(s, &tm_k, &tm_v, p, b, hk, split, tbase) && tid == 0) sa_raise(SA_ERR_TIMEOUT);
+    if (!decode_body<D, SINK>(s, &tm_k, &tm_v, p, b, hk, split, tbase) && tid == 0) sa_raise(SA_ERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 64);

@@ -121,6 +121,7 @@ SA_DEV void quant16(const float (&xt)[16], int f_lo, int f_hi, uint32_t& w0, uin
     off = 0;
     if (SEARCH && c0 != 0) {
         float best = err16(xt, c0, w0, w1);
+#pragma unroll 1
         for (int f = f_lo; f < f_hi; ++f) {
             int c = (int)c0 + f;
             if (f == 0 || c < 0 || c > 0x7E) continue;

@@ -459,14 +459,16 @@ sa_status sa_thrift_select(const void* q_dev, const void* k_dev, int B, int H, i
                                ws_bytes, stream);
 }
 
-sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,
-                      const uint8_t* k_codes_dev, const uint8_t* k_scales_dev, const float* k_g_dev,
-                      const uint8_t* v_codes_dev, const uint8_t* v_scales_dev, const float* v_g_dev, int B, int H,
-                      int N, int D, int causal, float sm_scale, const uint8_t* mask_dev, const void* q_bf16_dev,
-                      const void* k_bf16_dev, const void* v_bf16_dev, const float* k_mean_dev, float* out_dev,
-                      float* lse_dev, cudaStream_t stream)
+sa_status sa_attn_fwd_ex(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,
+                         const uint8_t* k_codes_dev, const uint8_t* k_scales_dev, const float* k_g_dev,
+                         const uint8_t* v_codes_dev, const uint8_t* v_scales_dev, const float* v_g_dev, int B, int H,
+                         int N, int D, int causal, float sm_scale, int p_mode, const uint8_t* mask_dev,
+                         const void* q_bf16_dev, const void* k_bf16_dev, const void* v_bf16_dev,
+                         const float* k_mean_dev, float* out_dev, float* lse_dev, cudaStream_t stream)
 {
     if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+    if (p_mode != SA_SCALE_MAX && p_mode != SA_SCALE_SEARCH) return SA_ERR_INVALID_ARG;
+    if (p_mode == SA_SCALE_SEARCH && mask_dev) return SA_ERR_UNSUPPORTED;
     if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
     if (N % 32) return SA_ERR_INVALID_ARG;
     if ((size_t)B * H * N == 0) return SA_OK;
@@ -522,24 +524,41 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
     const int nsm = sm_count();
     if (nsm <= 0) return SA_ERR_CUDA;
     const unsigned grid = (unsigned)(nitems < nsm ? nitems : nsm);  // persistent: one CTA per SM
-#define SA_ATTN_LAUNCH(DD, MX)                                                                              \
+#define SA_ATTN_LAUNCH(DD, MX, PS)                                                                          \
     do {                                                                                                    \
         const int smem = (int)sizeof(PpSmem<DD, MX>) + 1024;                                                \
         static PerDevice attr; /* set on a device's first call, outside any stream capture */              \
-        if (!allow_smem(attr, attn_fwd_pp_kernel<DD, MX>, smem)) return SA_ERR_CUDA;                        \
+        if (!allow_smem(attr, attn_fwd_pp_kernel<DD, MX, PS>, smem)) return SA_ERR_CUDA;                    \
         static PerDevice regs_ok; /* the kernel's register split must fit its launch allocation */         \
-        if (once_per_device(regs_ok, [] { return pp_regs_fit(attn_fwd_pp_kernel<DD, MX>) ? 1 : 0; }) <= 0)  \
+        if (once_per_device(regs_ok, [] { return pp_regs_fit(attn_fwd_pp_kernel<DD, MX, PS>) ? 1 : 0; }) <= 0) \
             return SA_ERR_UNSUPPORTED;                                                                      \
-        attn_fwd_pp_kernel<DD, MX><<<grid, kPpThreads, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);       \
+        attn_fwd_pp_kernel<DD, MX, PS><<<grid, kPpThreads, smem, stream>>>(tq, tk, tv, tqb, tkb, tvb, p);   \
     } while (0)
+    const bool ps = p_mode == SA_SCALE_SEARCH;
     if (D == 128) {
-        if (mixed) SA_ATTN_LAUNCH(128, true); else SA_ATTN_LAUNCH(128, false);
+        if (mixed) SA_ATTN_LAUNCH(128, true, false);
+        else if (ps) SA_ATTN_LAUNCH(128, false, true);
+        else SA_ATTN_LAUNCH(128, false, false);
     } else {
-        if (mixed) SA_ATTN_LAUNCH(64, true); else SA_ATTN_LAUNCH(64, false);
+        if (mixed) SA_ATTN_LAUNCH(64, true, false);
+        else if (ps) SA_ATTN_LAUNCH(64, false, true);
+        else SA_ATTN_LAUNCH(64, false, false);
     }
 #undef SA_ATTN_LAUNCH
     SA_CHECK_LAUNCH();
     return SA_OK;
+}
+
+sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,
+                      const uint8_t* k_codes_dev, const uint8_t* k_scales_dev, const float* k_g_dev,
+                      const uint8_t* v_codes_dev, const uint8_t* v_scales_dev, const float* v_g_dev, int B, int H,
+                      int N, int D, int causal, float sm_scale, const uint8_t* mask_dev, const void* q_bf16_dev,
+                      const void* k_bf16_dev, const void* v_bf16_dev, const float* k_mean_dev, float* out_dev,
+                      float* lse_dev, cudaStream_t stream)
+{
+    return sa_attn_fwd_ex(q_codes_dev, q_scales_dev, q_g_dev, k_codes_dev, k_scales_dev, k_g_dev, v_codes_dev,
+                          v_scales_dev, v_g_dev, B, H, N, D, causal, sm_scale, SA_SCALE_MAX, mask_dev, q_bf16_dev,
+                          k_bf16_dev, v_bf16_dev, k_mean_dev, out_dev, lse_dev, stream);
 }
 
 size_t sa_decode_workspace_size(int B, int Hq, int Hkv, int L, int D)
@@ -549,18 +568,25 @@ size_t sa_decode_workspace_size(int B, int Hq, int Hkv, int L, int D)
     return 256 + sa_align256((size_t)B * Hq * nsplit * (D + 2) * sizeof(float));
 }
 
-sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
-                               const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
-                               const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
-                               float* out_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream)
+sa_status sa_attn_decode_kvfp4_sink(const void* q_dev, const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                                    const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
+                                    const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
+                                    int sink_first, int sink_last, const void* k_sink_dev, const void* v_sink_dev,
+                                    const float* k_mean_dev, float* out_dev, void* ws_dev, size_t ws_bytes,
+                                    cudaStream_t stream)
 {
     if (B < 0 || Hq < 0 || Hkv <= 0 || L < 0) return SA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
     if (Hq % Hkv || Hq / Hkv > kDecN || L % 128) return SA_ERR_INVALID_ARG;
+    if (sink_first < 0 || sink_last < 0 || (long)(sink_first + (long)sink_last) * 128 > L) return SA_ERR_INVALID_ARG;
+    const bool sink = sink_first > 0 || sink_last > 0;
     if ((size_t)B * Hq == 0) return SA_OK;
     if (L == 0) return SA_ERR_INVALID_ARG;
     if (!q_dev || !k_codes_dev || !k_scales_dev || !k_g_dev || !v_codes_dev || !v_scales_dev || !v_g_dev ||
         !out_dev || !ws_dev)
+        return SA_ERR_INVALID_ARG;
+    if (sink && (!k_sink_dev || !v_sink_dev || !aligned16(k_sink_dev) || !aligned16(v_sink_dev) ||
+                 ((uintptr_t)k_mean_dev & 15u)))
         return SA_ERR_INVALID_ARG;
     if (!aligned16(q_dev) || !aligned16(k_codes_dev) || !aligned16(v_codes_dev) || !aligned16(k_scales_dev) ||
         !aligned16(v_scales_dev) || ((uintptr_t)ws_dev & 255u))
@@ -596,22 +622,52 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
     p.RTk = sa_cdiv(L, 128);
     p.CKv = sa_cdiv(L, 64);
     p.sm_scale = sm_scale;
+    if (sink) {
+        p.k_sink = (const uint16_t*)k_sink_dev;
+        p.v_sink = (const uint16_t*)v_sink_dev;
+        p.k_mean = k_mean_dev;
+        p.sink_first = sink_first;
+        p.sink_last = sink_last;
+        p.NS = 128 * (sink_first + sink_last);
+    }
     dim3 grid(nsplit, Hkv, B);
     if (D == 128) {
         const int smem = (int)sizeof(DecSmem<128>) + 1024;
-        static PerDevice attr;
-        if (!allow_smem(attr, decode_kernel<128>, smem)) return SA_ERR_CUDA;
-        decode_kernel<128><<<grid, 128, smem, stream>>>(tk, tv, p);
+        if (sink) {
+            static PerDevice attr;
+            if (!allow_smem(attr, decode_kernel<128, true>, smem)) return SA_ERR_CUDA;
+            decode_kernel<128, true><<<grid, 128, smem, stream>>>(tk, tv, p);
+        } else {
+            static PerDevice attr;
+            if (!allow_smem(attr, decode_kernel<128, false>, smem)) return SA_ERR_CUDA;
+            decode_kernel<128, false><<<grid, 128, smem, stream>>>(tk, tv, p);
+        }
     } else {
         const int smem = (int)sizeof(DecSmem<64>) + 1024;
-        static PerDevice attr;
-        if (!allow_smem(attr, decode_kernel<64>, smem)) return SA_ERR_CUDA;
-        decode_kernel<64><<<grid, 128, smem, stream>>>(tk, tv, p);
+        if (sink) {
+            static PerDevice attr;
+            if (!allow_smem(attr, decode_kernel<64, true>, smem)) return SA_ERR_CUDA;
+            decode_kernel<64, true><<<grid, 128, smem, stream>>>(tk, tv, p);
+        } else {
+            static PerDevice attr;
+            if (!allow_smem(attr, decode_kernel<64, false>, smem)) return SA_ERR_CUDA;
+            decode_kernel<64, false><<<grid, 128, smem, stream>>>(tk, tv, p);
+        }
     }
     SA_CHECK_LAUNCH();
     decode_combine_kernel<<<(unsigned)(B * Hq), 128, 0, stream>>>(part, nsplit, D, v_g_dev, out_dev);
     SA_CHECK_LAUNCH();
     return SA_OK;
+}
+
+sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                               const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
+                               const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
+                               float* out_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream)
+{
+    return sa_attn_decode_kvfp4_sink(q_dev, k_codes_dev, k_scales_dev, k_g_dev, v_codes_dev, v_scales_dev, v_g_dev, B,
+                                     Hq, Hkv, L, D, sm_scale, 0, 0, nullptr, nullptr, nullptr, out_dev, ws_dev,
+                                     ws_bytes, stream);
 }
 
 }  // extern "C"

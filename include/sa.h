@@ -266,6 +266,25 @@ sa_status sa_attn_fwd(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, c
                       float* lse_dev, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * sa_attn_fwd_ex -- sa_attn_fwd with the block rule of the requantised P
+ * chosen: p_mode SA_SCALE_MAX is sa_attn_fwd; SA_SCALE_SEARCH applies
+ * ScaleSearch to P ("Search Your Block Floating Point Scales!", "ScaleSearch":
+ * the same candidates as for Q, K and V, i.e. per 16 keys the scale codes
+ * c0 + f, f in [-2, 6), c0 = E4M3(max p~ / 6), on p~ = P~ * 2688, keeping the
+ * least squared error of p~, ties to the lower candidate in the order
+ * f = 0, -2, -1, 1, ..., 5).  The search costs about eight block encodings
+ * per 16 keys on the softmax's critical path.  SA_SCALE_SEARCH with a
+ * high-precision block mask returns SA_ERR_UNSUPPORTED; another p_mode
+ * returns SA_ERR_INVALID_ARG.  Other arguments and errors as sa_attn_fwd.
+ * ------------------------------------------------------------------------ */
+sa_status sa_attn_fwd_ex(const uint8_t* q_codes_dev, const uint8_t* q_scales_dev, const float* q_g_dev,
+                         const uint8_t* k_codes_dev, const uint8_t* k_scales_dev, const float* k_g_dev,
+                         const uint8_t* v_codes_dev, const uint8_t* v_scales_dev, const float* v_g_dev, int B, int H,
+                         int N, int D, int causal, float sm_scale, int p_mode, const uint8_t* mask_dev,
+                         const void* q_bf16_dev, const void* k_bf16_dev, const void* v_bf16_dev,
+                         const float* k_mean_dev, float* out_dev, float* lse_dev, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * sa_attn_decode_kvfp4 -- one query token per sequence over an NVFP4 KV
  * cache ("ScaleSearchAttention": the KV cache kept in 4 bits), grouped-query
  * heads (query head h reads kv head h / (Hq/Hkv)).  q is quantised like a Q
@@ -286,6 +305,39 @@ sa_status sa_attn_decode_kvfp4(const void* q_dev, const uint8_t* k_codes_dev, co
                                const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
                                const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
                                float* out_dev, void* ws_dev, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * sa_attn_decode_kvfp4_sink -- sa_attn_decode_kvfp4 over an attention-sink-
+ * aware mixed-precision cache ("Search Your Block Floating Point Scales!",
+ * "ScaleSearchAttention": the first and last blocks of the cache are kept at
+ * full precision, the middle ones in NVFP4).  Reading: a block is a 128-key
+ * cache tile and "full precision" is the raw bf16 cache.  The first
+ * sink_first and the last sink_last tiles of each (b, kv head) take the
+ * mixed-block arithmetic of sa_attn_fwd's high-precision blocks inside the
+ * same split-wise online softmax: score = q . (k - mean(K)) * sm_scale with
+ * the raw bf16 q and k (the mean only when K was smoothed), P rounded to
+ * bf16, raw bf16 V.  The NVFP4 codes of those tiles are not read.
+ *
+ *  sink_first,
+ *  sink_last       tiles kept at full precision at each end of the cache;
+ *                  (0, 0) is sa_attn_decode_kvfp4.  128 (sink_first +
+ *                  sink_last) <= L, otherwise SA_ERR_INVALID_ARG.
+ *  k_sink_dev,
+ *  v_sink_dev      bf16 [B, Hkv, 128 (sink_first + sink_last), D], 16-byte
+ *                  aligned: per (b, kv head) the first sink_first tiles of the
+ *                  cache, then its last sink_last tiles, keys ascending.
+ *  k_mean_dev      FP32 [B, Hkv, D], the channel means that smoothed the K
+ *                  cache (sa_quant_nvfp4's k_mean output), or NULL when K was
+ *                  quantised without smoothing.
+ * The other arguments, the workspace and the errors are those of
+ * sa_attn_decode_kvfp4.  Caller-owned buffers, none retained.
+ * ------------------------------------------------------------------------ */
+sa_status sa_attn_decode_kvfp4_sink(const void* q_dev, const uint8_t* k_codes_dev, const uint8_t* k_scales_dev,
+                                    const float* k_g_dev, const uint8_t* v_codes_dev, const uint8_t* v_scales_dev,
+                                    const float* v_g_dev, int B, int Hq, int Hkv, int L, int D, float sm_scale,
+                                    int sink_first, int sink_last, const void* k_sink_dev, const void* v_sink_dev,
+                                    const float* k_mean_dev, float* out_dev, void* ws_dev, size_t ws_bytes,
+                                    cudaStream_t stream);
 
 #ifdef __cplusplus
 }

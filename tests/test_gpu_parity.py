@@ -293,6 +293,55 @@ def test_attention_matches_oracle(name, shape, causal, mode, rows):
     print("  quality vs exact (oracle): cos %.6f relL1 %.4f" % quality(ref[:, :, :64], ex))
 
 
+# ------------------------------------------------------------------ ScaleSearch on P
+P_SEARCH_CASES = [
+    ("tiny", {}, True, "max", None),                   # every row compared
+    ("tiny", {"N": 416, "D": 128}, False, "search", None),  # ragged last tile, D = 128
+    ("tiny", {"N": 352}, True, "search", None),        # ragged, causal, D = 64
+    ("llm", {"B": 1, "H": 4}, True, "search", None),   # LLM shape, every row of 4 heads
+    ("llm", {}, True, "search", "sample"),             # the full LLM workload: Q, K, P, V all ScaleSearch
+]
+
+
+@pytest.mark.parametrize("name,shape,causal,mode,rows", P_SEARCH_CASES)
+def test_attention_p_search_matches_oracle(name, shape, causal, mode, rows):
+    """ScaleSearch on the requantised P (sa_attn_fwd_ex) against the oracle's
+    attention with P searched the same way."""
+    q, k, v = inputs(name, **shape)
+    B, H, N, D = q.shape
+    qg, kg, vg = (gpu_quant(x, r, mode=mode) for x, r in ((q, "q"), (k, "k"), (v, "v")))
+    og, lg = sa.sa_attn_fwd(qg, kg, vg, causal, want_lse=True, p_mode="search")
+    status_ok()
+    og, lg = og.cpu().numpy(), lg.cpu().numpy()
+    ss = mode == "search"
+    qo, ko, vo = orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss), orc.quantize(v, "v", search=ss)
+    rr = sample_rows(N) if rows == "sample" else None
+    ref, lse_ref = orc.attention(qo, ko, vo, causal, rows=rr, want_lse=True, p_search=True)
+    got = og if rr is None else og[:, :, rr]
+    lse_got = lg if rr is None else lg[:, :, rr]
+    check_close(got, ref, f"attn P-search {name}{shape} causal={causal} {mode}")
+    assert np.max(np.abs(lse_got - lse_ref)) < 1e-3
+    if rr is None:
+        # the searched P is a different requantisation: the max-scaled oracle is further away
+        ref_max = orc.attention(qo, ko, vo, causal)
+        d_search = np.abs(og - ref).mean()
+        d_max = np.abs(og - ref_max).mean()
+        print("  mean |gpu - oracle(P search)| %.3e, |gpu - oracle(P max)| %.3e" % (d_search, d_max))
+        assert d_search < d_max
+
+
+def test_attention_p_search_with_mask_is_unsupported():
+    q, k, v = inputs("tiny")
+    B, H, N, D = q.shape
+    qg, kg, vg = (gpu_quant(x, r) for x, r in ((q, "q"), (k, "k"), (v, "v")))
+    T = (N + 127) // 128
+    mask = torch.zeros(B, H, T, T, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        sa.sa_attn_fwd(qg, kg, vg, True, mask=mask, q_bf16=q.cuda(), k_bf16=k.cuda(), v_bf16=v.cuda(),
+                       p_mode="search")
+    status_ok()
+
+
 # ------------------------------------------------------------------ decode
 def run_decode(q, k, v):
     B, Hkv, L, D = k.shape
@@ -324,6 +373,71 @@ def test_decode_full_size_sampled():
     pairs = np.array(sorted(set(fixed) | {int(e) for e in extra}), np.int32)
     ref = orc.decode(q, ko, vo, pairs=pairs)
     check_close(og.reshape(-1, 128)[pairs], ref, "decode full")
+
+
+# ------------------------------------------------------------------ sink-aware decode cache
+def sink_cache(shape, seed=0):
+    """Decode inputs whose first and last keys carry extra score mass (the
+    attention-sink pattern): the first and last 8 keys of every head x3."""
+    q, k, v = wl.decode_inputs(seed=seed, **shape) if shape else wl.decode_inputs("decode", seed=seed)
+    k = k.float()
+    k[:, :, :8] *= 3.0
+    k[:, :, -8:] *= 3.0
+    return q, k.bfloat16(), v
+
+
+def run_decode_sink(q, k, v, tiles, smooth=True):
+    kg = gpu_quant(k, "k", smooth=smooth)
+    vg = gpu_quant(v, "v")
+    kd, vd = k.cuda(), v.cuda()
+    out = sa.sa_attn_decode_kvfp4(q.cuda(), kg, vg, sink_tiles=tiles, k_sink=sa.sink_tiles_of(kd, *tiles),
+                                  v_sink=sa.sink_tiles_of(vd, *tiles))
+    status_ok()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape,tiles,smooth", [
+    (dict(B=2, Hq=8, Hkv=2, L=8192, D=128), (1, 1), True),
+    (dict(B=2, Hq=8, Hkv=2, L=8192, D=128), (4, 36), True),   # the last tiles span two splits
+    (dict(B=1, Hq=4, Hkv=4, L=4096 + 384, D=64), (2, 3), True),
+    (dict(B=1, Hq=4, Hkv=4, L=4096 + 384, D=64), (1, 0), False),  # K not smoothed
+    (dict(B=3, Hq=8, Hkv=1, L=256, D=128), (1, 1), True),   # every tile at full precision
+    (dict(B=2, Hq=6, Hkv=2, L=1024, D=128), (0, 2), True),  # G = 3
+])
+def test_decode_sink_matches_oracle(shape, tiles, smooth):
+    q, k, v = sink_cache(shape)
+    og = run_decode_sink(q, k, v, tiles, smooth)
+    ko, vo = orc.quantize(k, "k", smooth=smooth), orc.quantize(v, "v")
+    ref = orc.decode(q, ko, vo, sink_tiles=tiles, k_bf16=k, v_bf16=v).reshape(og.shape)
+    check_close(og, ref, f"decode sink {shape} {tiles}")
+    # the full-precision tiles matter: the plain NVFP4 decode is measurably further away
+    plain = orc.decode(q, ko, vo).reshape(og.shape)
+    print("  |sink - plain| / max|O| = %.2e" % (np.max(np.abs(ref - plain)) / np.max(np.abs(ref))))
+
+
+def test_decode_sink_full_size_sampled():
+    """Decode workload (B32 Hq32 Hkv8 L32768 D128) with the first and last
+    tile at full precision; all outputs from the GPU, sampled (b, head)
+    pairs from the oracle."""
+    q, k, v = sink_cache(None)
+    tiles = (1, 1)
+    og = run_decode_sink(q, k, v, tiles)
+    ko, vo = orc.quantize(k, "k"), orc.quantize(v, "v")
+    pairs = np.array(sorted({0, 7, 32 * 9 + 4, 32 * 31 + 31} |
+                            {int(e) for e in np.random.default_rng(5).choice(32 * 32, size=20, replace=False)}),
+                     np.int32)
+    ref = orc.decode(q, ko, vo, pairs=pairs, sink_tiles=tiles, k_bf16=k, v_bf16=v)
+    check_close(og.reshape(-1, 128)[pairs], ref, "decode sink full")
+
+
+def test_decode_sink_none_is_plain_decode():
+    """sink_tiles = (0, 0) runs the plain NVFP4 decode (bit-identical)."""
+    q, k, v = wl.decode_inputs(B=2, Hq=8, Hkv=2, L=8192, D=128)
+    kg, vg = gpu_quant(k, "k"), gpu_quant(v, "v")
+    a = sa.sa_attn_decode_kvfp4(q.cuda(), kg, vg)
+    b = sa.sa_attn_decode_kvfp4(q.cuda(), kg, vg, sink_tiles=(0, 0))
+    status_ok()
+    assert torch.equal(a, b)
 
 
 # ------------------------------------------------------------------ mixed precision
