@@ -86,20 +86,64 @@ SA_DEV void encode16(const float (&xt)[16], uint32_t c, uint32_t& w0, uint32_t& 
     w1 = pack8_e2m1(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
 }
 
-// Squared error of a coded block: e_i = x~_i - v_i*s (v_i*s exact), two
-// interleaved fmaf accumulators, summed at the end.
+// The eight E2M1 codes of a word (byte k = elements 2k, 2k+1, low nibble
+// first) as exact floats: one hardware conversion per byte to an f16 pair,
+// then f16 -> f32 (every E2M1 value is exact in both).
+SA_DEV void e2m1x8_to_f32(uint32_t w, float (&v)[8])
+{
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t.reg .b16 l0, u0, l1, u1, l2, u2, l3, u3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %8;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+        "mov.b32 {l0, u0}, h0;\n\t"
+        "mov.b32 {l1, u1}, h1;\n\t"
+        "mov.b32 {l2, u2}, h2;\n\t"
+        "mov.b32 {l3, u3}, h3;\n\t"
+        "cvt.f32.f16 %0, l0;\n\t"
+        "cvt.f32.f16 %1, u0;\n\t"
+        "cvt.f32.f16 %2, l1;\n\t"
+        "cvt.f32.f16 %3, u1;\n\t"
+        "cvt.f32.f16 %4, l2;\n\t"
+        "cvt.f32.f16 %5, u2;\n\t"
+        "cvt.f32.f16 %6, l3;\n\t"
+        "cvt.f32.f16 %7, u3;\n\t}"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "r"(w));
+}
+
+// d_i = a_i * b_i + c_i for a pair (IEEE RN per lane, one instruction).
+SA_DEV void fma2_rn(float a0, float a1, float b0, float b1, float c0, float c1, float& d0, float& d1)
+{
+    asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// Squared error of a coded block: e_i = x~_i - v_i*s (v_i*s is exact, so one
+// rounded fma(-v_i, s, x~_i) gives it), two interleaved accumulators
+// a_(i mod 2) = fma(e_i, e_i, a_(i mod 2)) over i ascending, summed at the
+// end.  Elements 2k and 2k+1 share one paired instruction, lane 0 even.
 SA_DEV float err16(const float (&xt)[16], uint32_t c, uint32_t w0, uint32_t w1)
 {
-    float s = e4m3_to_f32(c);
+    const float s = e4m3_to_f32(c);
     float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-        uint32_t nib = ((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 15u;
-        float e = __fsub_rn(xt[i], __fmul_rn(e2m1_to_f32(nib), s));
-        if (i & 1)
-            a1 = __fmaf_rn(e, e, a1);
-        else
-            a0 = __fmaf_rn(e, e, a0);
+    for (int h = 0; h < 2; h++) {
+        float v[8];
+        e2m1x8_to_f32(h ? w1 : w0, v);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            float e0, e1;
+            fma2_rn(-v[2 * k], -v[2 * k + 1], s, s, xt[8 * h + 2 * k], xt[8 * h + 2 * k + 1], e0, e1);
+            fma2_rn(e0, e1, e0, e1, a0, a1, a0, a1);
+        }
     }
     return __fadd_rn(a0, a1);
 }
