@@ -9,13 +9,14 @@ Metric: FP4 attention TOPS = 4*B*H*N^2*D / t (causal halved), t = step time.
 The headline workload is the long-context mixed-precision prefill (B1 H32
 N65536 D128 causal, top 5% of blocks in bf16), the largest configuration that
 fits one GPU; the LLM prefill (max-scaling, ScaleSearch on Q, K and V, and
-ScaleSearch on Q, K, V and P), the video-shaped
+ScaleSearch on Q, K, V and P, and incoherence processing of Q and K before
+max-scaling), the video-shaped
 prefill and the NVFP4-KV decode (plain, and with the cache's first and last
 128-key tile at full precision) are measured in the same run and nested in the
 line under "workloads".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME [--only]]
-                  [--mode max|search|psearch|sink] [--impl ours|reference]
+                  [--mode max|search|psearch|ip|sink] [--impl ours|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica (the path has no
 cross-GPU exchange), timing is the max over ranks, value is the job total.
@@ -158,6 +159,10 @@ class Path:
         w, st = self.w, self.st
         if w.kind == "decode":
             return  # the KV cache is quantised once, before timing (it is a cache)
+        if self.mode == "ip":  # Q and K through incoherence processing, V as usual
+            st["q"], st["k"], st["r"] = sa.sa_quant_nvfp4_ip(self.q, self.k, st["signs"])
+            st["v"] = sa.sa_quant_nvfp4(self.v, "v", out=st.get("v"))
+            return
         # Q, K (smoothed) and V in two launches: statistics, then quantisation
         st["qkv"] = sa.sa_quant_nvfp4_qkv(self.q, self.k, self.v, smooth=True, mode=prepass_mode(self.mode),
                                           out=st.get("qkv"))
@@ -179,6 +184,8 @@ class Path:
         return st["o"]
 
     def setup(self):
+        if self.mode == "ip":
+            self.st["signs"] = torch.from_numpy(ip_signs(self.w.D)).to(self.q.device)
         if self.w.kind == "decode":
             self.st["kc"] = sa.sa_quant_nvfp4(self.k, "k")
             self.st["vc"] = sa.sa_quant_nvfp4(self.v, "v")
@@ -221,15 +228,24 @@ def p_mode(mode):
     return "search" if mode == "psearch" else "max"
 
 
+def ip_signs(D, seed=7):
+    """Random signs of the incoherence rotation (mode "ip")."""
+    import numpy as np
+
+    return np.where(np.random.default_rng(seed).random(D) < 0.5, -1, 1).astype(np.int8)
+
+
 def sink_tiles(mode):
     """Decode mode "sink": the first and the last 128-key tile of the cache
     at full precision (the attention-sink-aware mixed-precision cache)."""
     return (1, 1) if mode == "sink" else (0, 0)
 
 
-def kernels_per_step(w):
+def kernels_per_step(w, mode="max"):
     if w.kind == "decode":
         return 3  # q amax, split kernel, combine
+    if mode == "ip":
+        return 6 + 2 + 1  # K mean (2) + rotation sums, r, amax, quantisation; V amax + quantisation; attention
     n = 2 + 1  # fused pre-pass: statistics + quantisation of Q, K, V; attention
     if w.thrift_bp:
         n += 3  # pool, score, top-k
@@ -277,7 +293,12 @@ def cpu_sample_step(w, mode, q, k, v, tiles):
     ss = prepass_mode(mode) == "search"
     N, D = w.N, w.D
     t0 = time.perf_counter()
-    qo, ko, vo = orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss), orc.quantize(v, "v", search=ss)
+    if mode == "ip":
+        qi, ki, _ = orc.incoherence(q, k, ip_signs(D), orc.quantize(k, "k").k_mean)
+        qo, ko, vo = orc.quantize_rows_f32(qi), orc.quantize_rows_f32(ki), orc.quantize(v, "v")
+    else:
+        qo, ko, vo = (orc.quantize(q, "q", search=ss), orc.quantize(k, "k", search=ss),
+                      orc.quantize(v, "v", search=ss))
     mask = None
     if w.thrift_bp:
         mask, _ = orc.thrift_select(q, k, w.causal, w.thrift_bp)
@@ -381,7 +402,8 @@ def traffic_of(w, kname, args):
 
 def config_of(w, mode):
     c = {"workload": w.description, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "causal": w.causal,
-         "scale_mode": prepass_mode(mode), "p_scale_mode": p_mode(mode), "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
+         "scale_mode": prepass_mode(mode), "p_scale_mode": p_mode(mode),
+         "incoherence_processing": mode == "ip", "l2": "flushed between steps (256 MiB write)", "parallelism": "replicas",
          "launch": "CUDA graphs (pre-pass graph + attention graph per step)"}
     if w.kind == "decode":
         c["Hkv"] = w.Hkv
@@ -466,7 +488,7 @@ def measure(w, mode, args, dev, pg, world, flush, want_e2e=True):
                 "algorithmic_bytes": attn_algorithmic_bytes(w), "ms_per_launch": ms_attn}
         value = whole_job_tops(world, flops, ms)
     out = {"value": value, "ms_per_step": ms, "config": config_of(w, mode), "roofline": roof,
-           "gpu_launches": kernels_per_step(w) * args.steps, "clocks": clk.summary(), "wall_s": t_wall}
+           "gpu_launches": kernels_per_step(w, mode) * args.steps, "clocks": clk.summary(), "wall_s": t_wall}
     if w.kind != "decode":
         ms_pre = ms - ms_attn  # the pre-pass (and selector) share of the step, between the graphs
         pb = prepass_bytes(w)
@@ -492,7 +514,7 @@ def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
     e2e_paths, houts = [], []
     for _ in range(2):
         pth = Path(w, mode, torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-        pth.st.update({kk: path.st[kk] for kk in ("kc", "vc", "ks", "vs") if kk in path.st})
+        pth.st.update({kk: path.st[kk] for kk in ("kc", "vc", "ks", "vs", "signs") if kk in path.st})
         e2e_paths.append(pth)
         houts.append(torch.empty(path.st["o"].shape, dtype=torch.float32).pin_memory())
 
@@ -550,8 +572,8 @@ def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
 # largest configuration that fits one GPU (the long-context mixed prefill);
 # the others are measured in the same run and nested in the line.
 HEADLINE = ("longctx", "max")
-OTHERS = [("llm", "max"), ("llm", "search"), ("llm", "psearch"), ("video", "search"), ("decode", "max"),
-          ("decode", "sink")]
+OTHERS = [("llm", "max"), ("llm", "search"), ("llm", "psearch"), ("llm", "ip"), ("video", "search"),
+          ("decode", "max"), ("decode", "sink")]
 
 
 def main():
@@ -560,13 +582,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=HEADLINE[0])
-    ap.add_argument("--mode", default=None, choices=["max", "search", "psearch", "sink"])
+    ap.add_argument("--mode", default=None, choices=["max", "search", "psearch", "ip", "sink"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only", action="store_true", help="measure the named workload alone (no nested workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (a smaller slice for ncu captures; not a bench line)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (a smaller slice for ncu captures; not a bench line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -576,10 +600,14 @@ def main():
     w = wl.WORKLOADS[args.workload]
     if args.mode is None:
         args.mode = "search" if w.scale_modes == ("search",) else "max"
-    if args.batch is not None:
+    if args.batch is not None or args.heads is not None:
         import dataclasses
 
-        w = dataclasses.replace(w, B=args.batch, description=w.description + f" (batch {args.batch} slice)")
+        B = w.B if args.batch is None else args.batch
+        H = w.H if args.heads is None else args.heads
+        if w.kind == "decode" and H % w.Hkv:
+            raise SystemExit("--heads must be a multiple of the workload's kv heads")
+        w = dataclasses.replace(w, B=B, H=H, description=w.description + f" (slice B{B} H{H})")
         args.only = True
 
     if args.impl == "reference":

@@ -76,6 +76,9 @@ def lib():
         L.sa_attn_decode_kvfp4_sink.restype = I
         L.sa_attn_fwd_ex.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, P, P, P, P, P, P, P]
         L.sa_attn_fwd_ex.restype = I
+        L.sa_quant_ip_workspace_size.argtypes, L.sa_quant_ip_workspace_size.restype = [I, I, I, I], Z
+        L.sa_quant_nvfp4_ip.argtypes = [P, P, I, I, I, I, P, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, Z, P]
+        L.sa_quant_nvfp4_ip.restype = I
         _lib = L
     return _lib
 
@@ -292,6 +295,41 @@ def sa_thrift_select_ex(q, k, causal: bool, frac_bp: int = 500, per_row: bool = 
            L.sa_thrift_select_ex(_ptr(q), _ptr(k), _ptr(k_mean), B, H, N, D, int(causal), int(frac_bp),
                                  int(per_row), _ptr(mask), _ptr(nsel), _ptr(ws), ws_bytes, _stream(stream)))
     return mask, nsel
+
+
+def sa_quant_nvfp4_ip(q, k, signs, smooth: bool = True, mode: str = "max", f_lo: int = -2, f_hi: int = 6,
+                      ss_offsets: bool = False, stream=None):
+    """Incoherence processing of bf16 q, k [B,H,N,D] (CUDA) and the NVFP4
+    pre-pass of the results (include/sa.h, sa_quant_nvfp4_ip).  signs: int8
+    [D] of +-1 on the same device.  Returns (Q' NVFP4Tensor, K' NVFP4Tensor,
+    r FP32 [B,H,D]); both tensors use the Q/K layout (role "q" for Q', "k"
+    for K', whose k_mean is the smoothing mean or None)."""
+    import torch
+
+    _bf16("q", q, 4)
+    B, H, N, D = q.shape
+    _bf16("k", k, 4, (B, H, N, D))
+    _tensor("signs", signs, torch.int8, 1, (D,))
+    m = _mode(mode)
+    L = lib()
+    outs = []
+    for role in ("q", "k"):
+        codes = _empty(L.sa_codes_bytes(B, H, N, D, 0), q.device)
+        scales = _empty(L.sa_scales_bytes(B, H, N, D, 0), q.device)
+        g = torch.empty(2, dtype=torch.float32, device=q.device)
+        km = torch.empty(B, H, D, dtype=torch.float32, device=q.device) if (role == "k" and smooth) else None
+        off = torch.empty(max(B * H * N * D // 16, 1), dtype=torch.int8, device=q.device) if ss_offsets else None
+        outs.append(NVFP4Tensor(codes, scales, g, role, (B, H, N, D), km, off))
+    r = torch.empty(B, H, D, dtype=torch.float32, device=q.device)
+    ws_bytes = L.sa_quant_ip_workspace_size(B, H, N, D)
+    ws = _empty(ws_bytes, q.device)
+    oq, ok = outs
+    _check("sa_quant_nvfp4_ip",
+           L.sa_quant_nvfp4_ip(_ptr(q), _ptr(k), B, H, N, D, _ptr(signs), int(smooth), m, f_lo, f_hi,
+                               _ptr(oq.codes), _ptr(oq.scales), _ptr(oq.g), _ptr(ok.codes), _ptr(ok.scales),
+                               _ptr(ok.g), _ptr(ok.k_mean), _ptr(r), _ptr(oq.ss_off), _ptr(ok.ss_off), _ptr(ws),
+                               ws_bytes, _stream(stream)))
+    return oq, ok, r
 
 
 def sa_attn_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: NVFP4Tensor, causal: bool, sm_scale: float = 0.0, mask=None,

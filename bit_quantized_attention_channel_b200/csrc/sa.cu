@@ -10,6 +10,7 @@
 
 #include "attn_pp.cuh"
 #include "decode.cuh"
+#include "incoherence.cuh"
 #include "quant.cuh"
 #include "select.cuh"
 
@@ -276,6 +277,98 @@ sa_status sa_quant_nvfp4(const void* x_dev, int B, int H, int N, int D, sa_role 
         }
 #undef SA_QR
     }
+    SA_CHECK_LAUNCH();
+    return SA_OK;
+}
+
+size_t sa_quant_ip_workspace_size(int B, int H, int N, int D)
+{
+    if (B < 0 || H < 0 || N < 0 || D < 0) return 0;
+    return ip_ws_layout(nullptr, B, H, N, D).bytes;
+}
+
+sa_status sa_quant_nvfp4_ip(const void* q_dev, const void* k_dev, int B, int H, int N, int D,
+                            const int8_t* signs_dev, int smooth, sa_scale_mode mode, int f_lo, int f_hi,
+                            uint8_t* q_codes_dev, uint8_t* q_scales_dev, float* q_g_dev, uint8_t* k_codes_dev,
+                            uint8_t* k_scales_dev, float* k_g_dev, float* k_mean_dev, float* r_dev,
+                            int8_t* q_ss_off_dev, int8_t* k_ss_off_dev, void* ws_dev, size_t ws_bytes,
+                            cudaStream_t stream)
+{
+    if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+    if (mode != SA_SCALE_MAX && mode != SA_SCALE_SEARCH) return SA_ERR_INVALID_ARG;
+    if (mode == SA_SCALE_SEARCH && !(f_lo >= -16 && f_lo <= 0 && f_hi > 0 && f_hi <= 16)) return SA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+    if (N % 16) return SA_ERR_INVALID_ARG;
+    if ((size_t)B * H * N == 0) return SA_OK;
+    if ((size_t)B * H > 65535) return SA_ERR_UNSUPPORTED;
+    if (!q_dev || !k_dev || !signs_dev || !q_codes_dev || !q_scales_dev || !q_g_dev || !k_codes_dev ||
+        !k_scales_dev || !k_g_dev || !ws_dev)
+        return SA_ERR_INVALID_ARG;
+    if (!aligned16(q_dev) || !aligned16(k_dev) || ((uintptr_t)q_codes_dev & 7u) || ((uintptr_t)k_codes_dev & 7u) ||
+        ((uintptr_t)ws_dev & 255u) || ((uintptr_t)k_mean_dev & 15u))
+        return SA_ERR_INVALID_ARG;
+    IpWs w = ip_ws_layout(ws_dev, B, H, N, D);
+    if (ws_bytes < w.bytes) return SA_ERR_WORKSPACE;
+    const size_t BH = (size_t)B * H;
+    const int T = sa_cdiv(N, kTile);
+    if (cudaMemsetAsync(w.amax, 0, 16, stream) != cudaSuccess) return SA_ERR_CUDA;
+    float* kmean = k_mean_dev ? k_mean_dev : w.kst.kmean;
+    if (smooth) {
+        dim3 g1(sa_cdiv(T, 256 / (D / 2)), (unsigned)BH);
+        if (D == 128)
+            kstats_kernel<128><<<g1, 256, 0, stream>>>((const uint32_t*)k_dev, N, T, w.kst.psum, w.kst.pmax,
+                                                        w.kst.pmin);
+        else
+            kstats_kernel<64><<<g1, 256, 0, stream>>>((const uint32_t*)k_dev, N, T, w.kst.psum, w.kst.pmax,
+                                                       w.kst.pmin);
+        SA_CHECK_LAUNCH();
+        kfinal_kernel<<<(unsigned)BH, 128, 0, stream>>>(w.kst.psum, w.kst.pmax, w.kst.pmin, N, T, D, kmean,
+                                                         w.amax + 2);
+        SA_CHECK_LAUNCH();
+    }
+    IpParams p{};
+    p.x[0] = (const uint16_t*)q_dev;
+    p.x[1] = (const uint16_t*)k_dev;
+    p.k_mean = smooth ? kmean : nullptr;
+    p.signs = signs_dev;
+    p.hn = (float)(1.0 / std::sqrt((double)D));
+    p.N = N;
+    p.T = T;
+    p.part[0] = w.part[0];
+    p.part[1] = w.part[1];
+    p.r = w.r;
+    p.r_out = r_dev;
+    p.amax = w.amax;
+    IpOut o{};
+    o.codes[0] = q_codes_dev;
+    o.codes[1] = k_codes_dev;
+    o.scales[0] = q_scales_dev;
+    o.scales[1] = k_scales_dev;
+    o.g[0] = q_g_dev;
+    o.g[1] = k_g_dev;
+    o.ss_off[0] = q_ss_off_dev;
+    o.ss_off[1] = k_ss_off_dev;
+    o.f_lo = f_lo;
+    o.f_hi = f_hi;
+    const dim3 grid3((unsigned)T, (unsigned)BH, 2);
+    const bool ss = mode == SA_SCALE_SEARCH;
+#define SA_IP(DD)                                                                                          \
+    do {                                                                                                   \
+        const int smem = 128 * (DD + 1) * (int)sizeof(float);                                              \
+        static PerDevice attr;                                                                             \
+        if (!allow_smem(attr, ip_sums_kernel<DD>, smem)) return SA_ERR_CUDA;                               \
+        ip_sums_kernel<DD><<<grid3, 128, smem, stream>>>(p);                                               \
+        SA_CHECK_LAUNCH();                                                                                 \
+        ip_r_kernel<<<(unsigned)BH, DD, 0, stream>>>(p, DD);                                               \
+        SA_CHECK_LAUNCH();                                                                                 \
+        ip_amax_kernel<DD><<<grid3, 128, 0, stream>>>(p);                                                  \
+        SA_CHECK_LAUNCH();                                                                                 \
+        if (ss) ip_quant_kernel<DD, true><<<grid3, 128, 0, stream>>>(p, o);                                \
+        else ip_quant_kernel<DD, false><<<grid3, 128, 0, stream>>>(p, o);                                  \
+    } while (0)
+    if (D == 128) SA_IP(128);
+    else SA_IP(64);
+#undef SA_IP
     SA_CHECK_LAUNCH();
     return SA_OK;
 }

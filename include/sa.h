@@ -235,6 +235,48 @@ sa_status sa_thrift_select_ex(const void* q_dev, const void* k_dev, const float*
                               void* ws_dev, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * sa_quant_nvfp4_ip -- incoherence processing of Q and K, then their NVFP4
+ * pre-pass ("Search Your Block Floating Point Scales!", "ScaleSearchAttention",
+ * 비일관성 처리 (IP) 및 크기 감소: a Hadamard rotation with random signs, as in
+ * QuIP#, and a linear pair Q' = Q R^-T, K' = K R that keeps every score).
+ * Reading: Q~ = Q H S, K~ = (K - mu) H S (H the orthonormal Sylvester
+ * Hadamard matrix, S = diag(signs), mu the K channel mean when smooth), R
+ * diagonal with r_c = (sum_t q~_tc^2 / sum_t k~_tc^2)^(1/4) (1 when a sum is
+ * 0), Q' = Q~ R^-1, K' = K~ R; Q'K'^T = Q (K - mu)^T.  Arithmetic: the
+ * rotation in FP32 as the fast Walsh-Hadamard butterfly, then times
+ * fl32(1/sqrt(D)) and the sign; the sums of squares in FP64 (rows ascending
+ * inside 128-row tiles, then tiles ascending); r in FP64; Q' = fl32(y / r),
+ * K' = fl32(y r).  Q' and K' are each quantised like a Q tensor (own tensor
+ * scale g = amax/2688, 16-channel blocks, max-scaling or ScaleSearch, no
+ * further smoothing) into the Q/K layouts of sa_quant_nvfp4; the attention
+ * consumes them unchanged (sa_attn_fwd with V quantised as usual).
+ *
+ *  q_dev, k_dev    bf16 [B,H,N,D], 16-byte aligned; D = 64 or 128;
+ *                  N % 16 == 0; B*H <= 65535.
+ *  signs_dev       int8 [D] of +1 / -1 (device memory; a negative entry is -1).
+ *  smooth          1: subtract the K channel mean before the rotation.
+ *  mode, f_lo,
+ *  f_hi            block rule, as sa_quant_nvfp4.
+ *  q_* / k_*       codes, scale atoms and {g, 1/g} of Q' and of K', sized and
+ *                  laid out as sa_quant_nvfp4's role-Q outputs.
+ *  k_mean_dev      FP32 [B,H,D] receives mu when smooth (may be NULL).
+ *  r_dev           FP32 [B,H,D] receives fl32(r) (may be NULL).
+ *  q_ss_off_dev,
+ *  k_ss_off_dev    int8 [B,H,N,D/16] ScaleSearch offsets, or NULL.
+ *  ws_dev          sa_quant_ip_workspace_size() bytes, 256-byte aligned.
+ * Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED (D, B*H), SA_ERR_WORKSPACE;
+ * inf/NaN in the rotated values sets SA_ERR_NONFINITE in the device status.
+ * Caller-owned buffers, none retained.
+ * ------------------------------------------------------------------------ */
+size_t sa_quant_ip_workspace_size(int B, int H, int N, int D);
+sa_status sa_quant_nvfp4_ip(const void* q_dev, const void* k_dev, int B, int H, int N, int D,
+                            const int8_t* signs_dev, int smooth, sa_scale_mode mode, int f_lo, int f_hi,
+                            uint8_t* q_codes_dev, uint8_t* q_scales_dev, float* q_g_dev, uint8_t* k_codes_dev,
+                            uint8_t* k_scales_dev, float* k_g_dev, float* k_mean_dev, float* r_dev,
+                            int8_t* q_ss_off_dev, int8_t* k_ss_off_dev, void* ws_dev, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * sa_attn_fwd -- NVFP4 attention forward (prefill).
  * "Search Your Block Floating Point Scales!", "ScaleSearchAttention /
  * 네이티브 NVFP4 실행": Q K^T and P V as block-scaled FP4 tensor-core MMAs

