@@ -26,8 +26,9 @@
 //                 TMEM lane quadrant w % 4 (query rows 32(w%4)..+31) and the
 //                 key half h = ((w - 4) / 4) % 2 (columns 64h..64h+63).  The
 //                 two halves of a row meet once per key tile, through shared
-//                 memory and a 64-thread named barrier, to agree on the row
-//                 max; each half then computes its four 16-key block scales
+//                 memory and an mbarrier of the quadrant's two warps (a
+//                 bounded wait), to agree on the row max; each half then
+//                 computes its four 16-key block scales
 //                 (one 32-bit scale word of P), its 64 codes and the rescale
 //                 of its half of [O | l].
 // Every SM sub-partition (warps w with equal w % 4) runs two softmax warps of
@@ -337,6 +338,56 @@ __device__ __noinline__ float pp_bf16_p_row(uint8_t* prow, uint32_t s_col, int s
         }
         *reinterpret_cast<uint4*>(prow + ((cc ^ swz) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
+    return ls;
+}
+
+// The softmax side of one bf16 block, out of line (rare, and kept out of the
+// NVFP4 loop's instruction footprint): wait until O is free (o_done, when this
+// tile had a P V before) and the shared bf16 P buffer is granted, write this
+// half row's P, release S, then bring this half's columns of [O | l] to the new
+// max (o_half: its first O column; l_col: the l column when this half keeps l,
+// else 0): on the tile's first key tile l starts at 0, later O and l are
+// rescaled by alpha when any row's max moved; finally hand P to the P V
+// issuer.  Returns the half row's sum of P (units of 2688 / g_V), or -1 when a
+// wait gave up.
+__device__ __noinline__ float pp_bf16_tile(uint64_t* o_done, uint32_t od_parity, uint64_t* pb_grant,
+                                           uint32_t pg_parity, uint64_t* s_free, uint64_t* p_full,
+                                           volatile int* abort, long long lim, uint8_t* prow, uint32_t s_col,
+                                           int swz, int kbase, bool edge, int N, bool causal, int row, float crow,
+                                           float cb, float msub, float kappa, bool first, float alpha,
+                                           uint32_t o_half, int hd, uint32_t l_col)
+{
+    if ((o_done && !pp_wait(o_done, od_parity, abort, lim)) || !pp_wait(pb_grant, pg_parity, abort, lim))
+        return -1.0f;
+    tc_fence_after();
+    const float ls = pp_bf16_p_row(prow, s_col, swz, kbase, edge, N, causal, row, crow, cb, msub, kappa);
+    tc_fence_before();
+    __syncwarp();
+    const bool lead = (threadIdx.x & 31) == 0;
+    if (lead) mbar_arrive(s_free);  // S is read
+    if (first) {
+        if (l_col) tmem_st1(l_col, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
+    } else if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+        for (int c = 0; c < hd; c += 32) {
+            float o[32];
+            tmem_ld32(o_half + c, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int i2 = 0; i2 < 32; i2++) o[i2] *= alpha;
+            tmem_st32(o_half + c, o);
+        }
+        if (l_col) {
+            const float lv = tmem_ld1_sync(l_col);
+            tmem_st1(l_col, lv * alpha);
+        }
+    }
+    tmem_wait_st();
+    fence_proxy_async();
+    tc_fence_before();
+    __syncwarp();
+    if (lead) mbar_arrive(p_full);
     return ls;
 }
 
@@ -845,11 +896,11 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                 const int kbase = u * 128 + 64 * h;
                 const bool edge = (p.causal && u == tq) || (u * 128 + 128 > p.N);  // keys to mask
                 if (edge) {
+                    // the masked keys (key >= N, or key > row when causal) are a suffix
+                    // of this half: keep the first nv
+                    const int nv = min(p.N, p.causal ? row + 1 : p.N) - kbase;
 #pragma unroll
-                    for (int i2 = 0; i2 < 64; i2++) {
-                        const int key = kbase + i2;
-                        if (key >= p.N || (p.causal && key > row)) sv[i2] = -INFINITY;
-                    }
+                    for (int i2 = 0; i2 < 64; i2++) sv[i2] = i2 < nv ? sv[i2] : -INFINITY;
                 }
                 float bmax[4];
 #pragma unroll
@@ -875,21 +926,19 @@ __global__ void __launch_bounds__(kPpThreads, 1) attn_fwd_pp_kernel(const __grid
                     // at a time (no array of packed P held across the waits).  O is free
                     // once this tile's previous P V finished; the shared bf16 P buffer
                     // once the bf16 block before this one (either tile) finished its P V.
-                    if ((k > 0 && !pp_wait(&s.o_done[x], (k - 1) & 1, abort, lim)) ||
-                        !pp_wait(&s.pb_grant[x], nb & 1, abort, lim)) {
+                    const float ls = pp_bf16_tile(k > 0 ? &s.o_done[x] : nullptr, (k - 1) & 1, &s.pb_grant[x], nb & 1,
+                                                  &s.s_free[x], &s.p_full[x], abort, lim,
+                                                  s.pb[h] + (r >> 3) * 1024 + (r & 7) * 128,
+                                                  tbase + lane_off + PP_S + 64 * h, r & 7, kbase, edge, p.N,
+                                                  p.causal != 0, row, crow, cb, msub, kappa, u == 0, alpha,
+                                                  o_col + HD * h, HD, h == 1 ? o_col + 128 : 0u);
+                    if (ls < 0.0f) {
                         ok = false;
                         break;
                     }
                     nb++;
-                    tc_fence_after();
-                    const float ls = pp_bf16_p_row(s.pb[h] + (r >> 3) * 1024 + (r & 7) * 128,
-                                                   tbase + lane_off + PP_S + 64 * h, r & 7, kbase, edge, p.N,
-                                                   p.causal != 0, row, crow, cb, msub, kappa);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.s_free[x]);  // S is read
                     lb = lb * alpha + ls;
-                    if (u == 0 && h == 1) tmem_st1(o_col + 128, 0.0f);  // l starts at 0 (no NVFP4 P V yet)
+                    continue;  // the bf16 tile is complete (P handed over)
                 } else {
                     const float lm = kLog2_2688 - msub;
                     uint32_t scw = 0;

@@ -282,6 +282,23 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int bhk = b * p.Hkv + hk;
 
+    // full-precision tiles of this split: start their K and V on the way to L2
+    // now, ahead of their turn in the key loop
+    if constexpr (SINK) {
+        if (tid < 2) {
+            const int t0 = split * (kSplit / 128), t1 = min(t0 + kSplit / 128, p.RTk);
+            for (int kt = t0; kt < t1; kt++) {
+                int sr = -1;
+                if (kt < p.sink_first)
+                    sr = kt * 128;
+                else if (kt >= p.RTk - p.sink_last)
+                    sr = (p.sink_first + kt - (p.RTk - p.sink_last)) * 128;
+                if (sr < 0) continue;
+                const uint16_t* base = (tid ? p.v_sink : p.k_sink) + ((size_t)(b * p.Hkv + hk) * p.NS + sr) * D;
+                bulk_prefetch_l2(base, 128 * D * 2);
+            }
+        }
+    }
     // ---- quantise the group's query rows (q^T operand + its scale atom)
     {
         float g, inv_g;

@@ -87,6 +87,13 @@ SA_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// Bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
+// ahead of use, asynchronously (no completion to wait for).
+SA_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 SA_DEV void tma_prefetch_desc(const CUtensorMap* map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
