@@ -51,7 +51,10 @@ L2_FLUSH_BYTES = 256 << 20
 # workload, scaled by the units of the full launch.  Keyed by workload, scale
 # mode and kernel; any other key (or a kernel changed since its capture)
 # reports null.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # decode_kernel<128>, batch-4 slice x 8 (155.0 MB read + write per slice launch)
+    ("decode", "max", "decode_kernel<128> + combine"): 1239.6e6,
+}
 
 
 def peaks():
@@ -393,11 +396,11 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def traffic_of(w, kname, args):
+def traffic_of(w, mode, kname, args):
     """Measured DRAM bytes per launch for the full workload, else None."""
-    if args.batch is not None:
+    if args.batch is not None or args.heads is not None:
         return None
-    return MEASURED_TRAFFIC.get((w.name, args.mode if w.kind != "decode" else "max", kname))
+    return MEASURED_TRAFFIC.get((w.name, mode, kname))
 
 
 def config_of(w, mode):
@@ -473,7 +476,7 @@ def measure(w, mode, args, dev, pg, world, flush, want_e2e=True):
     if w.kind == "decode":
         gbs = hbm_bytes_decode(w, mode) / (ms_attn * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": kname, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                "peak_source": f"{src} copy bandwidth", "traffic": traffic_of(w, kname, args),
+                "peak_source": f"{src} copy bandwidth", "traffic": traffic_of(w, mode, kname, args),
                 "traffic_unit": "DRAM bytes per launch (ncu, batch slice scaled)", "ms_per_launch": ms_attn,
                 "algorithmic_bytes": hbm_bytes_decode(w, mode)}
         value = whole_job_tops(world, flops, ms)
@@ -482,7 +485,7 @@ def measure(w, mode, args, dev, pg, world, flush, want_e2e=True):
         roof = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak,
                 "peak_source": f"{src} bf16 {bf16} TFLOP/s x 4 (FP4/bf16 nominal ratio)",
-                "traffic": traffic_of(w, kname, args),
+                "traffic": traffic_of(w, mode, kname, args),
                 "traffic_unit": "DRAM bytes per launch (ncu, batch slice scaled; the FP32 output's write-back "
                                 "that leaves L2 after the kernel ends is not in the kernel's count)",
                 "algorithmic_bytes": attn_algorithmic_bytes(w), "ms_per_launch": ms_attn}
