@@ -341,21 +341,21 @@ __device__ __noinline__ float pp_bf16_p_row(uint8_t* prow, uint32_t s_col, int s
     return ls;
 }
 
-// The softmax side of one bf16 block, out of line (rare, and kept out of the
-// NVFP4 loop's instruction footprint): wait until O is free (o_done, when this
-// tile had a P V before) and the shared bf16 P buffer is granted, write this
+// The softmax side of one bf16 block, inline (a call site in the softmax loop
+// slowed the NVFP4 tiles more than the code it moved out saved; the P row
+// below it stays a call): wait until O is free (o_done, when this tile had a
+// P V before) and the shared bf16 P buffer is granted, write this
 // half row's P, release S, then bring this half's columns of [O | l] to the new
 // max (o_half: its first O column; l_col: the l column when this half keeps l,
 // else 0): on the tile's first key tile l starts at 0, later O and l are
 // rescaled by alpha when any row's max moved; finally hand P to the P V
 // issuer.  Returns the half row's sum of P (units of 2688 / g_V), or -1 when a
 // wait gave up.
-__device__ __noinline__ float pp_bf16_tile(uint64_t* o_done, uint32_t od_parity, uint64_t* pb_grant,
-                                           uint32_t pg_parity, uint64_t* s_free, uint64_t* p_full,
-                                           volatile int* abort, long long lim, uint8_t* prow, uint32_t s_col,
-                                           int swz, int kbase, bool edge, int N, bool causal, int row, float crow,
-                                           float cb, float msub, float kappa, bool first, float alpha,
-                                           uint32_t o_half, int hd, uint32_t l_col)
+SA_DEV float pp_bf16_tile(uint64_t* o_done, uint32_t od_parity, uint64_t* pb_grant, uint32_t pg_parity,
+                          uint64_t* s_free, uint64_t* p_full, volatile int* abort, long long lim, uint8_t* prow,
+                          uint32_t s_col, int swz, int kbase, bool edge, int N, bool causal, int row, float crow,
+                          float cb, float msub, float kappa, bool first, float alpha, uint32_t o_half, int hd,
+                          uint32_t l_col)
 {
     if ((o_done && !pp_wait(o_done, od_parity, abort, lim)) || !pp_wait(pb_grant, pg_parity, abort, lim))
         return -1.0f;
