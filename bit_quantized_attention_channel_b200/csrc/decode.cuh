@@ -33,6 +33,8 @@
 // NVFP4 units: O += (2688 P_b) (V / g_V), l += 2688 P_b.
 #pragma once
 
+#include <cstddef>
+
 #include "attn.cuh"
 #include "quant.cuh"
 
@@ -65,6 +67,7 @@ struct DecSmem {
     uint8_t vsf[2 * 512];
     alignas(16) uint8_t qsf[D / 64 * 512];
     uint8_t psf[2 * 512];
+    alignas(16) uint16_t pb16[kDecN * 128];  // bf16 P of a full-precision tile, [head][key]
     float rcp[128];    // reciprocals of the E4M3 scale values
     float lg2sc[128];  // log2 of each nonzero E4M3 scale value
     float lred[4][kDecN];  // per-warp partial sums of the dequantised P
@@ -76,6 +79,21 @@ struct DecSmem {
     uint64_t mma_bar;
     uint32_t tmem_slot;
 };
+
+// A full-precision tile stages 128 D bytes across the K stage and the start of
+// the V stage, which must be adjacent.
+static_assert(offsetof(DecSmem<128>, v) == 128 * 128 / 2 && offsetof(DecSmem<64>, v) == 128 * 64 / 2,
+              "K and V stages are adjacent");
+// ... and keeps the group's raw q (G <= 8 rows of D bf16) and the K channel means
+// (D floats) in the bytes of the NVFP4 tile's P and K / V scale atoms, adjacent too.
+template <int D>
+constexpr bool dec_scratch_fits()
+{
+    return offsetof(DecSmem<D>, ksf) == offsetof(DecSmem<D>, p) + sizeof(DecSmem<D>::p) &&
+           offsetof(DecSmem<D>, vsf) == offsetof(DecSmem<D>, ksf) + sizeof(DecSmem<D>::ksf) &&
+           sizeof(DecSmem<D>::p) + sizeof(DecSmem<D>::ksf) + sizeof(DecSmem<D>::vsf) >= kDecN * D * 2 + D * 4;
+}
+static_assert(dec_scratch_fits<128>() && dec_scratch_fits<64>(), "raw q and K means fit the NVFP4 tile's scratch");
 
 // TMEM columns (64 allocated)
 constexpr uint32_t DM_S = 0, DM_O = 8, DM_SFK = 24, DM_SFQ = 32, DM_SFV = 40, DM_SFP = 48;
@@ -98,78 +116,96 @@ struct DecParams {
     int sink_first, sink_last, NS;
 };
 
-// One full-precision cache tile: thread tid holds key tid for the scores and
-// channel tid for P·V.  sv receives q.(k - mu) per head (h < G; padding
-// heads 0).  pbuf: 128 G floats of shared memory for P_b.
+// Full-precision tiles go through shared memory in halves of 64 keys (128 D
+// bytes: the K stage and the first bytes of the V stage, which that tile does
+// not use; rows D.. of the V stage, zero for D = 64, stay untouched), by
+// 16-byte cp.async copies.  K rows are stored with their 16-byte chunks
+// swizzled by the row (chunk c at c ^ (row mod D/8)) so that the score loop
+// below reads without bank conflicts; V rows are stored plain.
 template <int D>
-SA_DEV void dec_sink_scores(const DecParams& p, int b, int hk, int srow, float (&sv)[kDecN])
+SA_DEV void dec_stage_half(uint8_t* stage, const uint16_t* src, bool swz)
 {
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
     const int tid = threadIdx.x;
-    const size_t kv = (size_t)b * p.Hkv + hk;
-    const uint4* krow = reinterpret_cast<const uint4*>(p.k_sink + (kv * p.NS + srow + tid) * D);
-    const float* mu = p.k_mean ? p.k_mean + kv * D : nullptr;
-    const uint16_t* qg = p.q + ((size_t)b * p.Hq + (size_t)hk * p.G) * D;
+#pragma unroll
+    for (int j = 0; j < 64 * CPR / 128; j++) {
+        const int idx = tid + 128 * j, row = idx / CPR, c = idx % CPR;
+        const int pc = swz ? (c ^ (row & (CPR - 1))) : c;
+        cp_async16(smem_u32(stage + row * (2 * D) + pc * 16), src + (size_t)row * D + c * 8);
+    }
+    cp_async_commit();
+}
+
+// Scores of one staged half: threads 2k and 2k + 1 take key k's two halves of
+// the channels, sv = q.(k - mu) per head (h < G; padding heads 0), summed
+// over the pair so both hold the key's score.
+template <int D>
+SA_DEV void dec_sink_half_scores(const uint8_t* stage, const DecParams& p, const uint16_t* qs, const float* mu,
+                                 float (&sv)[kDecN])
+{
+    constexpr int CPR = D / 8, PC = CPR / 2;
+    const int tid = threadIdx.x, kk = tid >> 1, part = tid & 1;
 #pragma unroll
     for (int h = 0; h < kDecN; h++) sv[h] = 0.0f;
-#pragma unroll 2
-    for (int c = 0; c < D / 8; c++) {
-        const uint4 kr = __ldg(krow + c);
+#pragma unroll 1
+    for (int i = 0; i < PC; i++) {
+        const int c = part * PC + i;
+        const uint4 kr = *reinterpret_cast<const uint4*>(stage + kk * (2 * D) + ((c ^ (kk & (CPR - 1))) * 16));
         const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
         float kf[8];
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            kf[2 * i] = __uint_as_float(kw[i] << 16);
-            kf[2 * i + 1] = __uint_as_float(kw[i] & 0xFFFF0000u);
+        for (int e = 0; e < 4; e++) {
+            kf[2 * e] = __uint_as_float(kw[e] << 16);
+            kf[2 * e + 1] = __uint_as_float(kw[e] & 0xFFFF0000u);
         }
         if (mu) {
-            const float4 m0 = __ldg(reinterpret_cast<const float4*>(mu + 8 * c));
-            const float4 m1 = __ldg(reinterpret_cast<const float4*>(mu + 8 * c + 4));
+            const float4 m0 = *reinterpret_cast<const float4*>(mu + 8 * c);
+            const float4 m1 = *reinterpret_cast<const float4*>(mu + 8 * c + 4);
             kf[0] -= m0.x, kf[1] -= m0.y, kf[2] -= m0.z, kf[3] -= m0.w;
             kf[4] -= m1.x, kf[5] -= m1.y, kf[6] -= m1.z, kf[7] -= m1.w;
         }
 #pragma unroll
         for (int h = 0; h < kDecN; h++) {
             if (h >= p.G) break;
-            const uint4 qr = __ldg(reinterpret_cast<const uint4*>(qg + (size_t)h * D) + c);  // warp-uniform
+            const uint4 qr = *reinterpret_cast<const uint4*>(qs + h * D + 8 * c);
             const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w};
             float a = sv[h];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                a = fmaf(__uint_as_float(qw[i] << 16), kf[2 * i], a);
-                a = fmaf(__uint_as_float(qw[i] & 0xFFFF0000u), kf[2 * i + 1], a);
+            for (int e = 0; e < 4; e++) {
+                a = fmaf(__uint_as_float(qw[e] << 16), kf[2 * e], a);
+                a = fmaf(__uint_as_float(qw[e] & 0xFFFF0000u), kf[2 * e + 1], a);
             }
             sv[h] = a;
         }
     }
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) sv[h] += __shfl_xor_sync(0xffffffffu, sv[h], 1);
 }
 
-// O^T row d = tid (d < D) of a full-precision tile: sum over the 128 keys of
-// P_b[h][key] V[key][d] in FP32, returned per head.
+// P.V of one staged V half for channel d = tid (d < D): acc[h] += sum over its
+// 64 keys of P_b[h][key0 + key] V[key][d]; P_b from its bf16 bits.
 template <int D>
-SA_DEV void dec_sink_pv(const DecParams& p, int b, int hk, int srow, const float* pbuf, float (&acc)[kDecN])
+SA_DEV void dec_sink_half_pv(const uint8_t* stage, const uint16_t* pb, int key0, const DecParams& p,
+                             float (&acc)[kDecN])
 {
     const int tid = threadIdx.x;
-#pragma unroll
-    for (int h = 0; h < kDecN; h++) acc[h] = 0.0f;
     if (tid >= D) return;
-    const size_t kv = (size_t)b * p.Hkv + hk;
-    const uint16_t* vcol = p.v_sink + (kv * p.NS + srow) * D + tid;
+    const uint16_t* vcol = reinterpret_cast<const uint16_t*>(stage) + tid;
 #pragma unroll 1
-    for (int k0 = 0; k0 < 128; k0 += 8) {
+    for (int k0 = 0; k0 < 64; k0 += 8) {
         float vv[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) vv[i] = __uint_as_float((uint32_t)__ldg(vcol + (size_t)(k0 + i) * D) << 16);
+        for (int i = 0; i < 8; i++) vv[i] = __uint_as_float((uint32_t)vcol[(k0 + i) * D] << 16);
 #pragma unroll
         for (int h = 0; h < kDecN; h++) {
             if (h >= p.G) break;
+            const uint4 pw = *reinterpret_cast<const uint4*>(pb + h * 128 + key0 + k0);  // broadcast
+            const uint32_t w[4] = {pw.x, pw.y, pw.z, pw.w};
             float a = acc[h];
 #pragma unroll
-            for (int i = 0; i < 8; i += 4) {
-                const float4 pw = *reinterpret_cast<const float4*>(pbuf + h * 128 + k0 + i);  // broadcast
-                a = fmaf(pw.x, vv[i], a);
-                a = fmaf(pw.y, vv[i + 1], a);
-                a = fmaf(pw.z, vv[i + 2], a);
-                a = fmaf(pw.w, vv[i + 3], a);
+            for (int e = 0; e < 4; e++) {
+                a = fmaf(__uint_as_float(w[e] << 16), vv[2 * e], a);
+                a = fmaf(__uint_as_float(w[e] & 0xFFFF0000u), vv[2 * e + 1], a);
             }
             acc[h] = a;
         }
@@ -219,31 +255,74 @@ SA_DEV void dec_l_update(DecSmem<D>& s, const DecParams& p, int u)
     }
 }
 
-// The rest of a full-precision tile once its scores sv are known: running
-// max, P_b = bf16(2^(sv c - m)) into shared memory (the K tile's buffer,
-// unused by this tile), P·V on the CUDA cores, O^T = alpha O^T + kappa acc in
-// TMEM (kappa = 2688 / g_V, the accumulator's NVFP4 units), l += 2688 P_b.
+// One full-precision cache tile (rows srow.. of the compact bf16 copy): the
+// scores of both key halves, the running max, P_b = bf16(2^(t c - m)) into
+// shared memory (bf16 bits, exact), P.V on the CUDA cores in FP32, then
+// O^T = alpha O^T + kappa acc in TMEM (kappa = 2688 / g_V, the accumulator's
+// NVFP4 units) and l += 2688 P_b.  The first V half is copied while the max
+// and P are formed.
 template <int D>
-SA_DEV bool dec_sink_tile(DecSmem<D>& s, const DecParams& p, int b, int hk, int srow, int u,
-                          const float (&sv)[kDecN], float c, uint32_t tbase, uint32_t lane_off)
+SA_DEV bool dec_sink_tile(DecSmem<D>& s, const DecParams& p, int b, int hk, int srow, int u, float c,
+                          uint32_t tbase, uint32_t lane_off)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float m2[kDecN], alpha[kDecN];
-    dec_running_max(s, p, sv, c, m2, alpha);
-    float* pbuf = reinterpret_cast<float*>(s.k);  // [G][128] (4 KB <= the K tile's bytes)
+    const size_t kv = (size_t)b * p.Hkv + hk;
+    const uint16_t* ks = p.k_sink + (kv * p.NS + srow) * D;
+    const uint16_t* vs = p.v_sink + (kv * p.NS + srow) * D;
+    const uint16_t* qg = p.q + ((size_t)b * p.Hq + (size_t)hk * p.G) * D;
+    const float* mug = p.k_mean ? p.k_mean + kv * D : nullptr;
+    uint8_t* stage = s.k;
+    // the group's raw q rows and the K means, copied with the first K half
+    uint16_t* qs = reinterpret_cast<uint16_t*>(s.p);
+    float* mu = mug ? reinterpret_cast<float*>(s.p + kDecN * D * 2) : nullptr;
+    if (tid < p.G * D / 8) cp_async16(smem_u32(qs + 8 * tid), qg + 8 * tid);
+    if (mug && tid < D / 4) cp_async16(smem_u32(mu + 4 * tid), mug + 4 * tid);
+    {  // scores, running max and P (alpha is re-read from shared memory below)
+    float sa[kDecN], sb[kDecN];
+    dec_stage_half<D>(stage, ks, true);
+    cp_async_wait_all();
+    __syncthreads();
+    dec_sink_half_scores<D>(stage, p, qs, mu, sa);
+    __syncthreads();
+    dec_stage_half<D>(stage, ks + 64 * D, true);
+    cp_async_wait_all();
+    __syncthreads();
+    dec_sink_half_scores<D>(stage, p, qs, mu, sb);
+    __syncthreads();
+    dec_stage_half<D>(stage, vs, false);  // lands while the max and P are formed
+    float mx[kDecN], m2[kDecN], alpha[kDecN];
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) mx[h] = fmaxf(sa[h], sb[h]);
+    dec_running_max(s, p, mx, c, m2, alpha);
+    const int kk = tid >> 1;
+    const bool lead = (tid & 1) == 0;  // the even thread of a key pair writes its P
 #pragma unroll
     for (int h = 0; h < kDecN; h++) {
         if (h >= p.G) break;
-        const float pb = __bfloat162float(__float2bfloat16_rn(ex2f(fmaf(sv[h], c, -m2[h]))));
-        pbuf[h * 128 + tid] = pb;
-        float pv = pb * 2688.0f;  // exact: 8 significant bits times 21 * 2^7
+        const __nv_bfloat16 pa = __float2bfloat16_rn(ex2f(fmaf(sa[h], c, -m2[h])));
+        const __nv_bfloat16 pb = __float2bfloat16_rn(ex2f(fmaf(sb[h], c, -m2[h])));
+        if (lead) {
+            s.pb16[h * 128 + kk] = __bfloat16_as_ushort(pa);
+            s.pb16[h * 128 + 64 + kk] = __bfloat16_as_ushort(pb);
+        }
+        // each P_b times 2688 is exact (8 significant bits times 21 * 2^7)
+        float pv = lead ? __bfloat162float(pa) * 2688.0f + __bfloat162float(pb) * 2688.0f : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) pv += __shfl_xor_sync(0xffffffffu, pv, o);
         if (lane == 0) s.lred[warp][h] = pv;
     }
+    }
+    cp_async_wait_all();
     __syncthreads();
     float acc[kDecN];
-    dec_sink_pv<D>(p, b, hk, srow, pbuf, acc);
+#pragma unroll
+    for (int h = 0; h < kDecN; h++) acc[h] = 0.0f;
+    dec_sink_half_pv<D>(stage, s.pb16, 0, p, acc);
+    __syncthreads();
+    dec_stage_half<D>(stage, vs + 64 * D, false);
+    cp_async_wait_all();
+    __syncthreads();
+    dec_sink_half_pv<D>(stage, s.pb16, 64, p, acc);
     const float kappa = 2688.0f / p.v_g[0];
     uint32_t r[kDecN];
     if (u > 0)
@@ -255,7 +334,7 @@ SA_DEV bool dec_sink_tile(DecSmem<D>& s, const DecParams& p, int b, int hk, int 
             : "memory");
 #pragma unroll
     for (int h = 0; h < kDecN; h++) {
-        const float o = u > 0 ? __uint_as_float(r[h]) * alpha[h] : 0.0f;
+        const float o = u > 0 ? __uint_as_float(r[h]) * s.alpha[h] : 0.0f;
         r[h] = __float_as_uint(fmaf(acc[h], kappa, o));
     }
     asm volatile(
@@ -263,7 +342,7 @@ SA_DEV bool dec_sink_tile(DecSmem<D>& s, const DecParams& p, int b, int hk, int 
         "tcgen05.wait::st.sync.aligned;" ::"r"(tbase + lane_off + DM_O),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
         : "memory");
-    fence_proxy_async();  // the K tile's buffer goes back to the tensor copies
+    fence_proxy_async();  // the staged and scratch bytes go back to the tensor copies
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -360,9 +439,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
             }
         }
         if (sink) {
-            float sv[kDecN];
-            dec_sink_scores<D>(p, b, hk, srow, sv);
-            if (!dec_sink_tile<D>(s, p, b, hk, srow, u, sv, c_sink, tbase, lane_off)) return false;
+            if (!dec_sink_tile<D>(s, p, b, hk, srow, u, c_sink, tbase, lane_off)) return false;
             continue;
         }
         if (tid == 0) {

@@ -87,6 +87,15 @@ SA_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 16-byte asynchronous copy global -> shared (through L2 only), grouped with
+// commit and waited for with wait_all by the issuing thread.
+SA_DEV void cp_async16(uint32_t dst_smem, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+SA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+SA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // Bring `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
 // ahead of use, asynchronously (no completion to wait for).
 SA_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes)
