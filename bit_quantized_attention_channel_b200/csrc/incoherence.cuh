@@ -14,7 +14,8 @@
 // Walsh-Hadamard butterfly (stages of span 1, 2, ..., D/2, (a, b) ->
 // (a + b, a - b)), then y_j = fl(t_j hn) s_j with hn = fl32(1/sqrt(D)); the
 // sums of squares in FP64, rows ascending inside each 128-row tile, then the
-// tiles ascending; r in FP64; Q' = fl32(y / r), K' = fl32(y r).  Q' and K'
+// tiles ascending; r and the reciprocal 1/r in FP64 (the pair is Q~ R^-1,
+// K~ R); Q' = fl32(y (1/r)), K' = fl32(y r).  Q' and K'
 // are then quantised like Q rows (own tensor scale, 16-channel blocks, no
 // further smoothing).
 //
@@ -40,7 +41,7 @@ struct IpParams {
     float hn;              // fl32(1 / sqrt(D))
     int N, T;
     double* part[2];       // [B*H, T, D] per-tile sums of squares
-    double* r;             // [B*H, D]
+    double* r;             // [B*H, 2, D]: r, then 1/r
     float* r_out;          // [B*H, D] or nullptr
     unsigned* amax;        // [2] FP32 bit patterns of amax(Q'), amax(K')
 };
@@ -125,20 +126,21 @@ __global__ void ip_r_kernel(const IpParams p, int D)
         b = __dadd_rn(b, p.part[1][(bh * p.T + tile) * D + c]);
     }
     const double r = (a > 0.0 && b > 0.0) ? __dsqrt_rn(__dsqrt_rn(__ddiv_rn(a, b))) : 1.0;
-    p.r[bh * D + c] = r;
+    p.r[bh * 2 * D + c] = r;
+    p.r[bh * 2 * D + D + c] = __ddiv_rn(1.0, r);
     if (p.r_out) p.r_out[bh * D + c] = __double2float_rn(r);
 }
 
-// Q' = fl32(y / r) (which = 0), K' = fl32(y r) (which = 1), in place.
-template <int D>
-SA_DEV void ip_balance(const IpParams& p, int which, size_t bh, float (&y)[D])
+// The balancing factors of tensor `which`: 1/r for Q' (which = 0), r for K'.
+SA_DEV const double* ip_factors(const IpParams& p, int which, size_t bh, int D)
 {
-    const double* r = p.r + bh * D;
-#pragma unroll
-    for (int j = 0; j < D; j++) {
-        const double rv = __ldg(r + j);
-        y[j] = __double2float_rn(which ? __dmul_rn((double)y[j], rv) : __ddiv_rn((double)y[j], rv));
-    }
+    return p.r + bh * 2 * D + (which ? 0 : D);
+}
+
+// Q' = fl32(y (1/r)), K' = fl32(y r) for one element.
+SA_DEV float ip_balance1(float y, const double* f, int j)
+{
+    return __double2float_rn(__dmul_rn((double)y, __ldg(f + j)));
 }
 
 // grid (T, B*H, 2), 128 threads.
@@ -156,11 +158,12 @@ __global__ void __launch_bounds__(128) ip_amax_kernel(const IpParams p)
     if (t < rows) {
         float y[D];
         ip_rotate_row<D>(p, which, bh, tile * 128 + t, sgn, y);
-        ip_balance<D>(p, which, bh, y);
+        const double* f = ip_factors(p, which, bh, D);
 #pragma unroll
         for (int j = 0; j < D; j++) {
-            bad |= !isfinite(y[j]);
-            m = fmaxf(m, fabsf(y[j]));
+            const float v = ip_balance1(y[j], f, j);
+            bad |= !isfinite(v);
+            m = fmaxf(m, fabsf(v));
         }
     }
     if (bad) sa_raise(SA_ERR_NONFINITE);
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(128) ip_quant_kernel(const IpParams p, const I
     if (t < rows) {
         float y[D];
         ip_rotate_row<D>(p, which, bh, tile * 128 + t, sgn, y);
-        ip_balance<D>(p, which, bh, y);
+        const double* f = ip_factors(p, which, bh, D);
         const size_t row = bh * p.N + (size_t)tile * 128 + t;
         uint2* codes = reinterpret_cast<uint2*>(o.codes[which]) + row * NB;
         uint32_t word = 0;
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(128) ip_quant_kernel(const IpParams p, const I
         for (int j = 0; j < NB; j++) {
             float xt[16];
 #pragma unroll
-            for (int i = 0; i < 16; i++) xt[i] = __fmul_rn(y[16 * j + i], inv_g);
+            for (int i = 0; i < 16; i++) xt[i] = __fmul_rn(ip_balance1(y[16 * j + i], f, 16 * j + i), inv_g);
             uint32_t c0, c1, sc;
             int off;
             quant16<SEARCH>(xt, o.f_lo, o.f_hi, c0, c1, sc, off, rcp);
@@ -250,7 +253,7 @@ static IpWs ip_ws_layout(void* base, int B, int H, int N, int D)
         off += sa_align256(BH * T * D * sizeof(double));
     }
     w.r = (double*)(p + off);
-    off += sa_align256(BH * D * sizeof(double));
+    off += sa_align256(BH * 2 * D * sizeof(double));
     w.bytes = off;
     return w;
 }

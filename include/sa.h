@@ -245,8 +245,8 @@ sa_status sa_thrift_select_ex(const void* q_dev, const void* k_dev, const float*
  * 0), Q' = Q~ R^-1, K' = K~ R; Q'K'^T = Q (K - mu)^T.  Arithmetic: the
  * rotation in FP32 as the fast Walsh-Hadamard butterfly, then times
  * fl32(1/sqrt(D)) and the sign; the sums of squares in FP64 (rows ascending
- * inside 128-row tiles, then tiles ascending); r in FP64; Q' = fl32(y / r),
- * K' = fl32(y r).  Q' and K' are each quantised like a Q tensor (own tensor
+ * inside 128-row tiles, then tiles ascending); r and 1/r in FP64;
+ * Q' = fl32(y (1/r)), K' = fl32(y r).  Q' and K' are each quantised like a Q tensor (own tensor
  * scale g = amax/2688, 16-channel blocks, max-scaling or ScaleSearch, no
  * further smoothing) into the Q/K layouts of sa_quant_nvfp4; the attention
  * consumes them unchanged (sa_attn_fwd with V quantised as usual).

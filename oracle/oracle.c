@@ -428,7 +428,8 @@ int orc_quant_rows_f32(const float* x, long rows, int D, int search, int f_lo, i
  * D/2, each pair (a, b) -> (a + b, a - b)), then y_j = fl(t_j * hn) * s_j with
  * hn = fl32(1/sqrt(D)); K's input x_i = fl32(k_i - mu_i).  The sums of
  * squares in FP64: rows ascending inside 128-row tiles, then the tile
- * partials ascending.  r in FP64; Q' = fl32(y / r), K' = fl32(y * r).
+ * partials ascending.  r in FP64; R^-1 as the diagonal of FP64 reciprocals
+ * 1/r (the pair is Q~ R^-1, K~ R); Q' = fl32(y * (1/r)), K' = fl32(y * r).
  *  q, k: bf16 [B, H, N, D], D a power of two; signs: D entries of +-1.
  *  q_out, k_out: FP32 [B, H, N, D]; r_out: FP32 [B, H, D].
  */
@@ -481,9 +482,10 @@ int orc_incoherence(const uint16_t* q, const uint16_t* k, const float* k_mean, i
                 b += pb;
             }
             double r = (a > 0.0 && b > 0.0) ? sqrt(sqrt(a / b)) : 1.0;
+            double rinv = 1.0 / r;
             r_out[(size_t)bh * D + j] = (float)r;
             for (int t = 0; t < N; t++) {
-                q_out[((size_t)bh * N + t) * D + j] = (float)((double)yq[(size_t)t * D + j] / r);
+                q_out[((size_t)bh * N + t) * D + j] = (float)((double)yq[(size_t)t * D + j] * rinv);
                 k_out[((size_t)bh * N + t) * D + j] = (float)((double)yk[(size_t)t * D + j] * r);
             }
         }
