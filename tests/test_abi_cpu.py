@@ -76,6 +76,29 @@ def test_rejects_bad_arguments_before_launch(L):
     assert L.sa_thrift_select(n, n, 1, 1, 256, 64, 1, 20000, n, n, n, 0, n) == 1
 
 
+def test_new_entry_points_reject_bad_arguments_before_launch(L):
+    n = None
+    # attention with a P block rule: unknown mode; ScaleSearch on P with a bf16 block mask
+    assert L.sa_attn_fwd_ex(*([n] * 9), 1, 1, 64, 64, 0, 0.0, 7, *([n] * 8)) == 1
+    mask = ctypes.c_void_p(16)  # never dereferenced: the call returns first
+    assert L.sa_attn_fwd_ex(*([n] * 9), 1, 1, 64, 64, 0, 0.0, 1, mask, *([n] * 7)) == 2
+    # sink decode: negative counts, more sink tiles than the cache holds, missing sink buffers
+    dec = [n] * 7
+    assert L.sa_attn_decode_kvfp4_sink(*dec, 1, 8, 2, 256, 128, 0.0, -1, 0, n, n, n, n, n, 0, n) == 1
+    assert L.sa_attn_decode_kvfp4_sink(*dec, 1, 8, 2, 256, 128, 0.0, 2, 1, n, n, n, n, n, 0, n) == 1
+    assert L.sa_attn_decode_kvfp4_sink(*dec, 1, 8, 2, 256, 128, 0.0, 1, 1, n, n, n, n, n, 0, n) == 1
+    # sink decode with (0, 0) and no work is the plain call's empty case
+    assert L.sa_attn_decode_kvfp4_sink(*dec, 0, 8, 2, 256, 128, 0.0, 0, 0, n, n, n, n, n, 0, n) == 0
+    # incoherence pre-pass: unsupported D, N % 16, bad ScaleSearch range, null signs
+    assert L.sa_quant_nvfp4_ip(n, n, 1, 1, 128, 96, n, 1, 0, -2, 6, *([n] * 11), 0, n) == 2
+    assert L.sa_quant_nvfp4_ip(n, n, 1, 1, 100, 64, n, 1, 0, -2, 6, *([n] * 11), 0, n) == 1
+    assert L.sa_quant_nvfp4_ip(n, n, 1, 1, 128, 64, n, 1, 1, 1, 6, *([n] * 11), 0, n) == 1
+    assert L.sa_quant_nvfp4_ip(n, n, 1, 1, 128, 64, n, 1, 0, -2, 6, *([n] * 11), 0, n) == 1
+    assert L.sa_quant_ip_workspace_size(1, 2, 256, 128) > L.sa_quant_workspace_size(1, 2, 256, 128, 1)
+    # selector variants: per-row budget out of range
+    assert L.sa_thrift_select_ex(n, n, n, 1, 1, 256, 64, 1, -1, 1, n, n, n, 0, n) == 1
+
+
 def test_scales_to_logical_roundtrip():
     import numpy as np
     import torch
