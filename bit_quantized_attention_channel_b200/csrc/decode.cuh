@@ -75,7 +75,8 @@ struct DecSmem {
     float red[4][kDecN];
     float mnew[kDecN];
     float alpha[kDecN];
-    uint64_t tma_bar;
+    uint64_t k_bar;  // K tile + K scale atoms landed
+    uint64_t v_bar;  // V tile + V scale atoms landed
     uint64_t mma_bar;
     uint32_t tmem_slot;
 };
@@ -411,7 +412,7 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     tc_fence_before();
     __syncthreads();
 
-    uint32_t tma_phase = 0, mma_phase = 0;
+    uint32_t kph = 0, vph = 0, mma_phase = 0;
     if (tid == 0) {
         tc_fence_after();
         for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFQ + 4 * kb, smem_u32(s.qsf + 512 * kb));
@@ -425,45 +426,73 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     const int nkeys = min(kSplit, p.L - key0);
     const int ntiles = nkeys / 128;
     const float c_sink = p.sm_scale * kLog2e;  // full-precision tiles: t = q.(k - mu) sm_scale log2(e)
+    // Row of tile u in the compact full-precision copy, or -1 for an NVFP4 tile.
+    auto sink_row = [&](int u) -> int {
+        if constexpr (SINK) {
+            const int kt = key0 / 128 + u;
+            if (kt < p.sink_first) return kt * 128;
+            if (kt >= p.RTk - p.sink_last) return (p.sink_first + kt - (p.RTk - p.sink_last)) * 128;
+        }
+        return -1;
+    };
+    // The K stage (with its scale atoms) and the V stage are loaded separately:
+    // the next tile's K as soon as this tile's Q K^T has read the K stage, its
+    // V as soon as this tile's P V has read the V stage, so each copy overlaps
+    // the rest of the tile (no extra shared memory).
+    auto load_k = [&](int kt) {
+        mbar_expect_tx(&s.k_bar, 128 * D / 2 + KB * 512);
+        tma_load_3d(s.k, tm_k, &s.k_bar, 0, kt * 128, bhk);
+        bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + kt) * KB * 512, KB * 512, &s.k_bar);
+    };
+    auto load_v = [&](int kt) {
+        mbar_expect_tx(&s.v_bar, D * 64 + 2 * 512);
+        tma_load_3d(s.v, tm_v, &s.v_bar, 0, kt * D, bhk);
+        bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * kt) * 512, 2 * 512, &s.v_bar);
+    };
+    bool kin = false, vin = false;  // this tile's K / V copies already issued (prefetched)
+    // before giving up, let the copies in flight land (bounded) so none writes
+    // shared memory after the CTA has left
+    auto drain = [&]() {
+        if (tid == 0) {
+            if (kin) mbar_wait(&s.k_bar, kph);
+            if (vin) mbar_wait(&s.v_bar, vph);
+        }
+        return false;
+    };
     for (int u = 0; u < ntiles; u++) {
         const int ktile = key0 / 128 + u;
-        bool sink = false;
-        int srow = 0;
-        if constexpr (SINK) {
-            if (ktile < p.sink_first) {
-                sink = true;
-                srow = ktile * 128;
-            } else if (ktile >= p.RTk - p.sink_last) {
-                sink = true;
-                srow = (p.sink_first + ktile - (p.RTk - p.sink_last)) * 128;
-            }
-        }
-        if (sink) {
+        const int srow = sink_row(u);
+        if (srow >= 0) {  // full-precision tile (no copy in flight: none is prefetched for it)
             if (!dec_sink_tile<D>(s, p, b, hk, srow, u, c_sink, tbase, lane_off)) return false;
             continue;
         }
+        // prefetch the next tile when it is NVFP4 (not in the kernel with full-precision
+        // tiles, whose register budget it would overrun)
+        const bool next = !SINK && u + 1 < ntiles;
         if (tid == 0) {
-            mbar_expect_tx(&s.tma_bar, 128 * D / 2 + KB * 512 + D * 64 + 2 * 512);
-            tma_load_3d(s.k, tm_k, &s.tma_bar, 0, ktile * 128, bhk);
-            bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + ktile) * KB * 512, KB * 512, &s.tma_bar);
-            tma_load_3d(s.v, tm_v, &s.tma_bar, 0, ktile * D, bhk);
-            bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * ktile) * 512, 2 * 512, &s.tma_bar);
+            if (!kin) load_k(ktile);
+            if (!vin) load_v(ktile);
         }
-        if (__syncthreads_or(!mbar_wait(&s.tma_bar, tma_phase))) return false;
-        tma_phase ^= 1;
+        kin = vin = true;
+        if (__syncthreads_or(!mbar_wait(&s.k_bar, kph))) return drain();
+        kph ^= 1;
+        kin = false;
         if (tid == 0) {
             tc_fence_after();
             for (int kb = 0; kb < KB; kb++) tc_cp_sf(tbase + DM_SFK + 4 * kb, smem_u32(s.ksf + 512 * kb));
-            for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFV + 4 * kb, smem_u32(s.vsf + 512 * kb));
             for (int kb = 0; kb < KB; kb++)
                 mma_fp4(tbase + DM_S, make_sdesc(smem_u32(s.k) + 32 * kb, KSBO, 16, KSW),
                         make_sdesc(smem_u32(s.q) + 32 * kb, KSBO, 16, KSW), idesc_fp4(128, kDecN),
                         tbase + DM_SFK + 4 * kb, tbase + DM_SFQ + 4 * kb, kb > 0);
             tc_commit(&s.mma_bar);
         }
-        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return drain();
         mma_phase ^= 1;
         tc_fence_after();
+        if (next) {  // the K stage is free: the next tile's K lands during this one
+            if (tid == 0) load_k(ktile + 1);
+            kin = true;
+        }
 
         // ---- scores of this thread's key for the 8 columns
         float sv[kDecN];
@@ -536,10 +565,13 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         }
         fence_proxy_async();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!mbar_wait(&s.v_bar, vph))) return drain();  // this tile's V has landed
+        vph ^= 1;
+        vin = false;
         dec_l_update(s, p, u);
         if (tid == 0) {
             tc_fence_after();
+            for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFV + 4 * kb, smem_u32(s.vsf + 512 * kb));
             for (int kb = 0; kb < 2; kb++) tc_cp_sf(tbase + DM_SFP + 4 * kb, smem_u32(s.psf + 512 * kb));
             for (int kb = 0; kb < 2; kb++) {
                 const uint64_t pd = make_sdesc(smem_u32(s.p) + 32 * kb, 512, 16, 4);
@@ -549,9 +581,13 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
             }
             tc_commit(&s.mma_bar);
         }
-        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return false;
+        if (__syncthreads_or(!mbar_wait(&s.mma_bar, mma_phase))) return drain();
         mma_phase ^= 1;
         tc_fence_after();
+        if (next) {  // the V stage is free: the next tile's V lands during its Q K^T
+            if (tid == 0) load_v(ktile + 1);
+            vin = true;
+        }
     }
 
     // ---- write this split's unnormalised O (lane = channel), l and m
@@ -589,7 +625,8 @@ __global__ void __launch_bounds__(128, 8) decode_kernel(const __grid_constant__ 
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&s.tma_bar, 1);
+        mbar_init(&s.k_bar, 1);
+        mbar_init(&s.v_bar, 1);
         mbar_init(&s.mma_bar, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
