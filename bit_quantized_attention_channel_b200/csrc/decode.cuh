@@ -362,6 +362,43 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int bhk = b * p.Hkv + hk;
 
+    const int key0 = split * kSplit;
+    const int nkeys = min(kSplit, p.L - key0);
+    const int ntiles = nkeys / 128;
+    const float c_sink = p.sm_scale * kLog2e;  // full-precision tiles: t = q.(k - mu) sm_scale log2(e)
+    // Row of tile u in the compact full-precision copy, or -1 for an NVFP4 tile.
+    auto sink_row = [&](int u) -> int {
+        if constexpr (SINK) {
+            const int kt = key0 / 128 + u;
+            if (kt < p.sink_first) return kt * 128;
+            if (kt >= p.RTk - p.sink_last) return (p.sink_first + kt - (p.RTk - p.sink_last)) * 128;
+        }
+        return -1;
+    };
+    // The K stage (with its scale atoms) and the V stage are loaded separately:
+    // the next tile's K as soon as this tile's Q K^T has read the K stage, its
+    // V as soon as this tile's P V has read the V stage, so each copy overlaps
+    // the rest of the tile (no extra shared memory).
+    auto load_k = [&](int kt) {
+        mbar_expect_tx(&s.k_bar, 128 * D / 2 + KB * 512);
+        tma_load_3d(s.k, tm_k, &s.k_bar, 0, kt * 128, bhk);
+        bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + kt) * KB * 512, KB * 512, &s.k_bar);
+    };
+    auto load_v = [&](int kt) {
+        mbar_expect_tx(&s.v_bar, D * 64 + 2 * 512);
+        tma_load_3d(s.v, tm_v, &s.v_bar, 0, kt * D, bhk);
+        bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * kt) * 512, 2 * 512, &s.v_bar);
+    };
+    bool kin = false, vin = false;  // this tile's K / V copies already issued (prefetched)
+    // the first tile's copies go out before q is quantised (they do not depend on it)
+    if (sink_row(0) < 0) {
+        if (tid == 0) {
+            load_k(key0 / 128);
+            load_v(key0 / 128);
+        }
+        kin = vin = true;
+    }
+
     // full-precision tiles of this split: start their K and V on the way to L2
     // now, ahead of their turn in the key loop
     if constexpr (SINK) {
@@ -422,34 +459,6 @@ SA_DEV bool decode_body(DecSmem<D>& s, const CUtensorMap* tm_k, const CUtensorMa
         s.mnew[tid] = tid < p.G ? -INFINITY : 0.0f;
         s.alpha[tid] = 1.0f;
     }
-    const int key0 = split * kSplit;
-    const int nkeys = min(kSplit, p.L - key0);
-    const int ntiles = nkeys / 128;
-    const float c_sink = p.sm_scale * kLog2e;  // full-precision tiles: t = q.(k - mu) sm_scale log2(e)
-    // Row of tile u in the compact full-precision copy, or -1 for an NVFP4 tile.
-    auto sink_row = [&](int u) -> int {
-        if constexpr (SINK) {
-            const int kt = key0 / 128 + u;
-            if (kt < p.sink_first) return kt * 128;
-            if (kt >= p.RTk - p.sink_last) return (p.sink_first + kt - (p.RTk - p.sink_last)) * 128;
-        }
-        return -1;
-    };
-    // The K stage (with its scale atoms) and the V stage are loaded separately:
-    // the next tile's K as soon as this tile's Q K^T has read the K stage, its
-    // V as soon as this tile's P V has read the V stage, so each copy overlaps
-    // the rest of the tile (no extra shared memory).
-    auto load_k = [&](int kt) {
-        mbar_expect_tx(&s.k_bar, 128 * D / 2 + KB * 512);
-        tma_load_3d(s.k, tm_k, &s.k_bar, 0, kt * 128, bhk);
-        bulk_load(s.ksf, p.k_sf + ((size_t)bhk * p.RTk + kt) * KB * 512, KB * 512, &s.k_bar);
-    };
-    auto load_v = [&](int kt) {
-        mbar_expect_tx(&s.v_bar, D * 64 + 2 * 512);
-        tma_load_3d(s.v, tm_v, &s.v_bar, 0, kt * D, bhk);
-        bulk_load(s.vsf, p.v_sf + ((size_t)bhk * p.CKv + 2 * kt) * 512, 2 * 512, &s.v_bar);
-    };
-    bool kin = false, vin = false;  // this tile's K / V copies already issued (prefetched)
     // before giving up, let the copies in flight land (bounded) so none writes
     // shared memory after the CTA has left
     auto drain = [&]() {
