@@ -52,8 +52,10 @@ L2_FLUSH_BYTES = 256 << 20
 # mode and kernel; any other key (or a kernel changed since its capture)
 # reports null.
 MEASURED_TRAFFIC = {
-    # decode_kernel<128>, batch-4 slice x 8 (154.9 MB read + write per slice launch)
-    ("decode", "max", "decode_kernel<128> + combine"): 1239.5e6,
+    # decode_kernel<128>, batch-4 slice x 8 (154.8 MB read + write per slice launch)
+    ("decode", "max", "decode_kernel<128> + combine"): 1238.2e6,
+    # attn_fwd_pp_kernel<128>, video 3-head slice x 8 (25.73 MB per slice launch)
+    ("video", "search", "attn_fwd_pp_kernel<128>"): 205.8e6,
     # attn_fwd_pp_kernel<128>, batch-1 slice x 2 (14.36 MB per slice launch)
     ("llm", "max", "attn_fwd_pp_kernel<128>"): 28.73e6,
     ("llm", "search", "attn_fwd_pp_kernel<128>"): 28.73e6,
