@@ -578,9 +578,9 @@ def measure_e2e(w, mode, args, dev, pg, flush, path, q, k, v):
     return {"ms": ms, "h2d": h2d, "d2h": houts[0].numel() * 4}
 
 
-# The workload BASELINE's metric is quoted on when nothing is named: the
-# largest configuration that fits one GPU (the long-context mixed prefill);
-# the others are measured in the same run and nested in the line.
+# The headline workload: the largest configuration that fits one GPU (the
+# long-context mixed prefill); the others are measured in the same run and
+# nested in the line.
 HEADLINE = ("longctx", "max")
 OTHERS = [("llm", "max"), ("llm", "search"), ("llm", "psearch"), ("llm", "ip"), ("video", "search"),
           ("decode", "max"), ("decode", "sink")]
