@@ -552,6 +552,22 @@ def test_incoherence_rotation_is_a_signed_orthonormal_hadamard():
     assert np.allclose(row, expect, rtol=1e-6, atol=0)
 
 
+def test_incoherence_without_smoothing_keeps_the_raw_scores():
+    """With no K mean the pair keeps Q K^T itself (the rotation and R cancel),
+    and a channel offset of K survives into the scores unchanged."""
+    q, k, signs, _ = _ip_case(seed=44)
+    qo, ko, _ = orc.incoherence(q, k, signs, None)
+    S = np.einsum("bhid,bhjd->bhij", q.double().numpy(), k.double().numpy())
+    S2 = np.einsum("bhid,bhjd->bhij", qo.astype(np.float64), ko.astype(np.float64))
+    assert np.abs(S2 - S).max() <= 1e-6 * np.abs(S).max()
+    # the smoothed pair differs from it by exactly the per-row offset q . mu
+    mu = orc.quantize(k, "k").k_mean.astype(np.float64)
+    qs, ks, _ = orc.incoherence(q, k, signs, orc.quantize(k, "k").k_mean)
+    S3 = np.einsum("bhid,bhjd->bhij", qs.astype(np.float64), ks.astype(np.float64))
+    off = np.einsum("bhid,bhd->bhi", q.double().numpy(), mu)[..., None]
+    assert np.abs((S - S3) - off).max() <= 2e-6 * np.abs(S).max()
+
+
 def test_incoherence_rotation_is_the_hadamard_product_within_fp32_rounding():
     """The FP32 butterfly equals the plain definition (x - mu) H S, H_ij =
     (-1)^popcount(i & j) / sqrt(D), evaluated in FP64 as a matrix product,
